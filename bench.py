@@ -1,0 +1,330 @@
+"""Benchmark of calibrated block-sparse attention on B200 (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload wan13b] [--impl reference]
+
+A step is one inference call of the hot path: sparse_attn_fwd over the workload's
+calibrated skip list (masks, skip lists and the longest-first schedule are built before
+inference and held in memory, as the method prescribes).  Inputs are resident in HBM when
+the timed region starts; Q/K/V/O of the default workload (Wan-1.3B shape: 12 heads x
+32760 tokens x 128) total 403 MB, larger than L2, so no flush is needed between steps.
+value = kept-only TFLOPS = 4 D sum_kept |I_i||J_j| / time, summed over ranks (each rank
+runs a replica: scaling "weak").  The same line carries the dense-equivalent TFLOPS, the
+roofline of the attention kernel against the measured bf16 peak, the speedup over this
+build's own kernel with an all-kept list, an end-to-end figure with host<->device copies
+in the timed region, the calibration pass (fused LSE + block energies, selection)
+measured on the same shapes, and the float64 oracle timed on a bounded sample on the
+host cores.  `--impl reference` times that oracle alone as the reference arm.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "sparse attn TFLOPS (kept-only & dense-equiv) + % BF16 TC peak at 30% density"
+UNIT = "TFLOPS"
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return {"bf16_tflops": d["bf16_tflops"], "bf16_tflops_sustained": d["bf16_tflops_sustained"],
+                "hbm_gbs": d["hbm_gbs"], "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0, "source": "fallback"}
+
+
+def kept_flops(mask: np.ndarray, N: int, D: int, B: int, repeat_heads=(), n_anchor=None) -> float:
+    """4 D sum over kept (i, j) of |I_i| |J_j| with real (ragged) block sizes; repeat heads
+    count their anchor-space rows."""
+    H, nq, nk = mask.shape
+    kc = np.array([min((j + 1) * B, N) - j * B for j in range(nk)], np.float64)
+    total = 0.0
+    for h in range(H):
+        Nq = n_anchor if (h in repeat_heads and n_anchor is not None) else N
+        nqh = (Nq + B - 1) // B
+        rows = np.array([min((i + 1) * B, Nq) - i * B for i in range(nqh)], np.float64)
+        total += float(rows @ (mask[h, :nqh].astype(np.float64) @ kc))
+    return 4.0 * D * total
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling during the timed region."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "50",
+                 "-i", self.gpu_id], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            time.sleep(0.3)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.1)
+            self.proc.terminate()
+            out, _ = self.proc.communicate(timeout=10)
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for l in getattr(self, "lines", []):
+            parts = [p.strip() for p in l.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for n, val in zip(names, parts[4:8]):
+                if val.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def _time_calls(fn, steps, warmup, torch):
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    st = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(st)
+    for _ in range(steps):
+        fn()
+    e1.record(st)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / steps
+
+
+def cpu_baseline(wl, q, k, v, mask, budget_s: float = 12.0):
+    """The float64 oracle on a bounded sample: whole query blocks of head 0 (kept keys only
+    enter the softmax), as many as fit in ~budget_s.  Returns kept-only TFLOPS."""
+    import oracle
+    from threadpoolctl import threadpool_info
+    s = wl.shape
+    B, D, N = s.block, s.D, s.N
+    scale = 1.0 / math.sqrt(D)
+    q0 = q[0:1].float().cpu().numpy().astype(np.float64)
+    k0 = k[0:1].float().cpu().numpy().astype(np.float64)
+    v0 = v[0:1].float().cpu().numpy().astype(np.float64)
+    kc = np.array([min((j + 1) * B, N) - j * B for j in range(s.nblk)], np.float64)
+    done, flops, t0 = 0, 0.0, time.perf_counter()
+    while time.perf_counter() - t0 < budget_s and done < s.nblk:
+        i = (done * 37) % s.nblk
+        oracle.sparse_attention(q0, k0, v0, scale, B, mask[0:1], q_blocks=[i])
+        rows = min((i + 1) * B, N) - i * B
+        flops += 4.0 * D * rows * float(mask[0, i].astype(np.float64) @ kc)
+        done += 1
+    dt = time.perf_counter() - t0
+    threads = max([t.get("num_threads", 1) for t in threadpool_info()] or [1])
+    return {"value": flops / dt / 1e12, "unit": UNIT, "cores": int(threads), "kind": "oracle",
+            "sample": f"{done} query blocks of head 0 at {wl.name} (N={N}, D={D}), {dt:.1f} s, "
+                      f"float64 NumPy on {os.cpu_count()} host cores"}
+
+
+def run_reference(args):
+    """Reference arm: the float64 oracle, as it stands, on the host cores (rank 0 only)."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import torch
+    from calibrated_block_sparse_calib_b200 import synth
+    wl = synth.WORKLOADS[args.workload]
+    q, k, v = synth.make_qkv(wl, heads=1)
+    mask = synth.make_head_masks(wl)[:1]
+    per_step = []
+    for _ in range(args.warmup):
+        cpu_baseline(wl, q, k, v, mask, budget_s=0.5)
+    for _ in range(args.steps):
+        per_step.append(cpu_baseline(wl, q, k, v, mask, budget_s=max(1.0, 60.0 / max(1, args.steps))))
+    val = statistics.mean(p["value"] for p in per_step)
+    line = {"impl": "reference", "metric": METRIC, "value": val, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": wl.name, "H": wl.shape.H, "N": wl.shape.N, "D": wl.shape.D,
+                       "block": wl.shape.block},
+            "cpu_baseline": {"value": val, "unit": UNIT, "cores": per_step[0]["cores"], "kind": "oracle",
+                             "sample": per_step[0]["sample"]},
+            "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="wan13b", choices=["wan13b", "wan14b720p", "mochi1"])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true", help="skip dense / e2e / calibration legs")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import torch.distributed as dist
+    from calibrated_block_sparse_calib_b200 import ops, synth
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local)
+    ops.lib()
+
+    wl = synth.WORKLOADS[args.workload]
+    s = wl.shape
+    B, D, N, H = s.block, s.D, s.N, s.H
+    q, k, v = synth.make_qkv(wl, device=dev)
+    mask_np = synth.make_head_masks(wl)
+    mask = torch.from_numpy(mask_np).to(dev)
+    bl = ops.BlockList.from_mask(mask, B)
+    rep = [h in wl.repeat_heads for h in range(H)]
+    stride = wl.repeat_stride
+    n_anchor = ops.anchor_count(s.F, s.Hl, s.Wl, s.n_text, stride) if any(rep) else None
+    out = torch.empty_like(q)
+    if any(rep):
+        call = lambda: ops.sparse_attn_fwd_repeat(q, k, v, bl, rep, s.F, s.Hl, s.Wl, s.n_text, stride, out=out)
+    else:
+        call = lambda: ops.sparse_attn_fwd(q, k, v, bl, out=out)
+    flops_kept = kept_flops(mask_np, N, D, B, tuple(h for h in range(H) if rep[h]), n_anchor)
+    flops_dense = 4.0 * N * N * D * H
+    density = flops_kept / flops_dense
+    ops.device_check()
+
+    # ---- timed region: K inference calls ----------------------------------------
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize()
+    gpu_uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    gpu_id = gpu_uuid if gpu_uuid.startswith("GPU-") else f"GPU-{gpu_uuid}"
+    st = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(gpu_id) as clk:
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        e0.record(st)
+        for _ in range(args.steps):
+            call()
+        e1.record(st)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+    ops.device_check()
+    ms = e0.elapsed_time(e1) / args.steps
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    value = flops_kept * world / (ms * 1e-3) / 1e12
+    peaks = _peaks()
+
+    extras = {}
+    if not args.no_extras:
+        # own dense kernel: same pipeline, all-kept list
+        full = torch.ones_like(mask)
+        bl_dense = ops.BlockList.from_mask(full, B)
+        ms_dense = _time_calls(lambda: ops.sparse_attn_fwd(q, k, v, bl_dense, out=out), 10, 3, torch)
+        extras["dense_kernel"] = {"ms": ms_dense, "tflops": flops_dense / (ms_dense * 1e-3) / 1e12,
+                                  "speedup_sparse_vs_dense": ms_dense / ms}
+        # end to end through the public API with host buffers
+        qh, kh, vh = (t.cpu().pin_memory() for t in (q, k, v))
+        oh = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
+        qd, kd, vd = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+
+        def e2e_step():
+            qd.copy_(qh, non_blocking=True)
+            kd.copy_(kh, non_blocking=True)
+            vd.copy_(vh, non_blocking=True)
+            if any(rep):
+                ops.sparse_attn_fwd_repeat(qd, kd, vd, bl, rep, s.F, s.Hl, s.Wl, s.n_text, stride, out=out)
+            else:
+                ops.sparse_attn_fwd(qd, kd, vd, bl, out=out)
+            oh.copy_(out, non_blocking=True)
+
+        ms_e2e = _time_calls(e2e_step, 10, 3, torch)
+        if world > 1:
+            t = torch.tensor([ms_e2e], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ms_e2e = float(t.item())
+        nb = q.numel() * q.element_size()
+        extras["e2e"] = {"value": flops_kept * world / (ms_e2e * 1e-3) / 1e12, "unit": UNIT,
+                         "h2d_bytes_per_step": 3 * nb, "d2h_bytes_per_step": nb, "ms_per_step": ms_e2e}
+        # calibration rows on the same shapes: fused LSE + energy pass and selection
+        if wl.name == "wan13b":
+            energy = ops.block_energy(q, k, B)
+            ms_energy = _time_calls(lambda: ops.block_energy(q, k, B, out=energy), 3, 2, torch)
+            msk = torch.empty(energy.shape, dtype=torch.uint8, device=dev)
+            ms_sel = _time_calls(lambda: ops.select_mask(energy, 0.95, out=msk), 20, 3, torch)
+            sel_bytes = energy.numel() * 4 + msk.numel()
+            extras["calibration"] = {
+                "energy_ms": ms_energy,
+                "energy_tflops_qk": 2 * 2.0 * N * N * D * H / (ms_energy * 1e-3) / 1e12,
+                "energy_exps_per_s": 2.0 * N * N * H / (ms_energy * 1e-3),
+                "select_ms": ms_sel, "select_gbs": sel_bytes / (ms_sel * 1e-3) / 1e9,
+                "select_frac_hbm": sel_bytes / (ms_sel * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                "tau": 0.95, "selected_density": float(msk.float().mean().item())}
+            ops.device_check()
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": wl.name, "H": H, "N": N, "D": D, "block": B, "density": round(density, 4),
+                   "repeat_heads": sum(rep), "parallelism": f"replicas{world}",
+                   "l2": "inputs larger than L2 (Q/K/V/O 403 MB), no flush"},
+        "dense_equiv_tflops": flops_dense * world / (ms * 1e-3) / 1e12,
+        "frac_of_bf16_peak": value / world / peaks["bf16_tflops"],
+        "roofline": {"bound": "tensor", "achieved": value / world, "peak": peaks["bf16_tflops"],
+                     "unit": "TFLOP/s", "frac": value / world / peaks["bf16_tflops"], "traffic": None,
+                     "peak_source": f"{peaks['source']} bf16 burst", "kernel": "attn_fwd_kernel<128,128,2,2>",
+                     "frac_of_sustained": value / world / peaks["bf16_tflops_sustained"]},
+        "gpu_launches": args.steps,
+        "clocks": clk.summary(),
+    }
+    if "e2e" in extras:
+        line["e2e"] = extras.pop("e2e")
+    line.update(extras)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl, q, k, v, mask_np)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,320 @@
+// C ABI of libcalibatt.so (declared in include/calibatt.h): argument validation, TMA
+// descriptor encoding, and kernel launches.  The library allocates no device memory;
+// its only state is the per-device status word in ptx.cuh and a few host-side caches
+// (the driver entry point, per-device capability and shared-memory attributes).
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <set>
+#include <utility>
+
+#include "calibatt.h"
+#include "ptx.cuh"
+#include "attn_fwd.cuh"
+#include "energy.cuh"
+#include "select.cuh"
+
+namespace {
+
+constexpr uint64_t kDefaultTimeoutNs = 4000000000ull;   // bounded device waits: 4 s
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+int cdiv(long long a, long long b) { return static_cast<int>((a + b - 1) / b); }
+
+cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+// sm_100 check, cached per device.
+calib_status check_device() {
+    static std::mutex mu;
+    static std::set<int> ok_devices;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return CALIB_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(mu);
+    if (ok_devices.count(dev)) return CALIB_OK;
+    int major = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+        return CALIB_ERR_CUDA;
+    if (major != 10) return CALIB_ERR_UNSUPPORTED;
+    ok_devices.insert(dev);
+    return CALIB_OK;
+}
+
+// Raise a kernel's dynamic shared-memory limit once per (kernel, device).
+calib_status ensure_smem(const void* fn, int bytes) {
+    static std::mutex mu;
+    static std::set<std::pair<const void*, int>> done;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return CALIB_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(mu);
+    if (done.count({fn, dev})) return CALIB_OK;
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+        return CALIB_ERR_CUDA;
+    done.insert({fn, dev});
+    return CALIB_OK;
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                   CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                   CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// 3-D bf16 view [H][N][D] of a contiguous tensor; box = 64 elements (128 B, the swizzle
+// span) x box_rows x 1, 128-byte swizzle, zero fill out of bounds.
+bool make_tmap(CUtensorMap* map, const void* base, int D, int N, int H, int box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(N),
+                                static_cast<cuuint64_t>(H)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(N) * D * 2};
+    const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+calib_status launch_status() {
+    return cudaGetLastError() == cudaSuccess ? CALIB_OK : CALIB_ERR_CUDA;
+}
+
+// ---- attention ---------------------------------------------------------------------
+template <int D, int BLK>
+calib_status launch_attn(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                         const calib::AttnParams& p, int grid, cudaStream_t st) {
+    constexpr int KST = 2, VST = 2;
+    using L = calib::AttnSmem<D, BLK, KST, VST>;
+    auto* fn = calib::attn_fwd_kernel<D, BLK, KST, VST>;
+    if (calib_status s = ensure_smem(reinterpret_cast<const void*>(fn), L::BYTES)) return s;
+    fn<<<grid, calib::kAttnThreads, L::BYTES, st>>>(tq, tk, tv, p);
+    return launch_status();
+}
+
+calib_status attn_common(const void* q, const void* k, const void* v, void* o, float* lse, int H, int N,
+                         int D, float scale, const calib_block_list* list, const uint32_t* repeat_bits,
+                         int F, int Hl, int Wl, int n_text, int stride, uint32_t flags, void* stream) {
+    if (!q || !k || !v || !o || !list || !list->row_ptr || !list->col_idx) return CALIB_ERR_INVALID;
+    if (flags & ~CALIB_ATTN_OUT_F32) return CALIB_ERR_INVALID;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return CALIB_ERR_INVALID;
+    if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return CALIB_ERR_INVALID;
+    if (H < 1 || N < 1 || !(scale > 0.f) || !std::isfinite(scale)) return CALIB_ERR_INVALID;
+    if (H > 1024 || static_cast<long long>(H) * N * D >= (1ll << 40)) return CALIB_ERR_INVALID;
+    const int B = list->block;
+    if (B != 64 && B != 128) return CALIB_ERR_INVALID;
+    if (D != 64 && D != 128) return CALIB_ERR_UNSUPPORTED;
+    const int nb = cdiv(N, B);
+    if (list->H != H || list->nq != nb || list->nk != nb || nb > 32767 || H > 32767) return CALIB_ERR_INVALID;
+    if (list->work && list->n_work < 0) return CALIB_ERR_INVALID;
+    if (calib_status s = check_device()) return s;
+    const int grid = list->work ? list->n_work : H * nb;
+    if (grid == 0) return CALIB_OK;
+
+    calib::AttnParams p{};
+    p.q = static_cast<const __nv_bfloat16*>(q);
+    p.o = static_cast<__nv_bfloat16*>(o);
+    p.lse = lse;
+    p.row_ptr = list->row_ptr;
+    p.col_idx = list->col_idx;
+    p.work = list->work;
+    p.H = H; p.N = N; p.nq = nb; p.nk = nb;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.F = F; p.Hl = Hl; p.Wl = Wl; p.n_text = n_text; p.stride = stride;
+    p.Ar = stride > 0 ? (Hl + stride - 1) / stride : 0;
+    p.n_anchor = F * p.Ar * Wl + n_text;
+    p.nq_anchor = cdiv(p.n_anchor, B);
+    for (int w = 0; w < 32; ++w) p.repeat_bits[w] = repeat_bits ? repeat_bits[w] : 0u;
+    p.out_f32 = (flags & CALIB_ATTN_OUT_F32) ? 1 : 0;
+    p.timeout_ns = kDefaultTimeoutNs;
+
+    CUtensorMap tq, tk, tv;
+    if (!make_tmap(&tq, q, D, N, H, calib::kTileM) || !make_tmap(&tk, k, D, N, H, B) ||
+        !make_tmap(&tv, v, D, N, H, B))
+        return CALIB_ERR_CUDA;
+    cudaStream_t st = as_stream(stream);
+    if (D == 128) return B == 128 ? launch_attn<128, 128>(tq, tk, tv, p, grid, st)
+                                  : launch_attn<128, 64>(tq, tk, tv, p, grid, st);
+    return B == 128 ? launch_attn<64, 128>(tq, tk, tv, p, grid, st) : launch_attn<64, 64>(tq, tk, tv, p, grid, st);
+}
+
+// ---- energy ------------------------------------------------------------------------
+template <int D, int BLK>
+calib_status launch_energy(const CUtensorMap& tq, const CUtensorMap& tk, const calib::EnergyParams& p,
+                           int grid, cudaStream_t st) {
+    constexpr int KST = 3;
+    using L = calib::EnergySmem<D, BLK, KST>;
+    auto* fn = calib::block_energy_kernel<D, BLK, KST>;
+    if (calib_status s = ensure_smem(reinterpret_cast<const void*>(fn), L::BYTES)) return s;
+    fn<<<grid, calib::kAttnThreads, L::BYTES, st>>>(tq, tk, p);
+    return launch_status();
+}
+
+int rows_grid(long long rows) { return static_cast<int>((rows + 3) / 4); }   // 4 warps per block
+
+}  // namespace
+
+extern "C" {
+
+const char* calib_status_string(calib_status s) {
+    switch (s) {
+        case CALIB_OK: return "CALIB_OK";
+        case CALIB_ERR_INVALID: return "CALIB_ERR_INVALID";
+        case CALIB_ERR_UNSUPPORTED: return "CALIB_ERR_UNSUPPORTED";
+        case CALIB_ERR_CUDA: return "CALIB_ERR_CUDA";
+        case CALIB_ERR_TIMEOUT: return "CALIB_ERR_TIMEOUT";
+    }
+    return "CALIB_ERR_UNKNOWN";
+}
+
+calib_status calib_device_check(void* stream) {
+    if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return CALIB_ERR_CUDA;
+    uint32_t v = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&v, calib::g_status, sizeof(v)) != cudaSuccess) return CALIB_ERR_CUDA;
+    if (v && cudaMemcpyToSymbol(calib::g_status, &zero, sizeof(zero)) != cudaSuccess) return CALIB_ERR_CUDA;
+    if (v & calib::STATUS_TIMEOUT) return CALIB_ERR_TIMEOUT;
+    if (v & calib::STATUS_BAD_ENERGY) return CALIB_ERR_INVALID;
+    return CALIB_OK;
+}
+
+calib_status calib_block_energy(const void* q, const void* k, const float* lse, int H, int N, int D, int block,
+                                float scale, const int32_t* q_rows, int n_q, float* energy, int accumulate,
+                                void* stream) {
+    if (!q || !k || !energy || !aligned16(q) || !aligned16(k)) return CALIB_ERR_INVALID;
+    if ((reinterpret_cast<uintptr_t>(energy) & 3u) || (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
+        return CALIB_ERR_INVALID;
+    if (H < 1 || N < 1 || !(scale > 0.f) || !std::isfinite(scale)) return CALIB_ERR_INVALID;
+    if (block != 64 && block != 128) return CALIB_ERR_INVALID;
+    if (D != 64 && D != 128) return CALIB_ERR_UNSUPPORTED;
+    const int Nq = q_rows ? n_q : N;
+    if (q_rows && n_q < 1) return CALIB_ERR_INVALID;
+    const int nq = cdiv(Nq, block), nk = cdiv(N, block);
+    if (static_cast<long long>(H) * nq > (1ll << 31) - 1) return CALIB_ERR_INVALID;
+    if (calib_status s = check_device()) return s;
+    calib::EnergyParams p{};
+    p.q = static_cast<const __nv_bfloat16*>(q);
+    p.q_rows = q_rows;
+    p.lse_in = lse;
+    p.energy = energy;
+    p.H = H; p.N = N; p.Nq = Nq; p.nq = nq; p.nk = nk;
+    p.accumulate = accumulate ? 1 : 0;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.timeout_ns = kDefaultTimeoutNs;
+    CUtensorMap tq, tk;
+    if (!make_tmap(&tq, q, D, N, H, calib::kTileM) || !make_tmap(&tk, k, D, N, H, block)) return CALIB_ERR_CUDA;
+    cudaStream_t st = as_stream(stream);
+    const int grid = H * nq;
+    if (D == 128) return block == 128 ? launch_energy<128, 128>(tq, tk, p, grid, st)
+                                      : launch_energy<128, 64>(tq, tk, p, grid, st);
+    return block == 128 ? launch_energy<64, 128>(tq, tk, p, grid, st) : launch_energy<64, 64>(tq, tk, p, grid, st);
+}
+
+calib_status calib_select_mask(const float* energy, int H, int nq, int nk, double tau, const uint8_t* force_keep,
+                               uint8_t* mask_out, int32_t* count_accum, void* stream) {
+    if (!energy || !mask_out) return CALIB_ERR_INVALID;
+    if (H < 1 || nq < 1 || nk < 1 || !(tau > 0.0) || !(tau <= 1.0)) return CALIB_ERR_INVALID;
+    if (nk > 32 * calib::kSelMaxPerLane) return CALIB_ERR_UNSUPPORTED;
+    if (static_cast<long long>(H) * nq * nk > (1ll << 31) - 1) return CALIB_ERR_INVALID;
+    if (calib_status s = check_device()) return s;
+    const int rows = H * nq;
+    calib::select_mask_kernel<<<rows_grid(rows), 128, 0, as_stream(stream)>>>(energy, rows, nq, nk, tau, force_keep,
+                                                                               mask_out, count_accum);
+    return launch_status();
+}
+
+calib_status calib_aggregate_masks(const int32_t* counts, int H, int nq, int nk, int n_inputs, int rho_num,
+                                   int rho_den, uint8_t* mask_out, void* stream) {
+    if (!counts || !mask_out) return CALIB_ERR_INVALID;
+    if (H < 1 || nq < 1 || nk < 1 || n_inputs < 1 || rho_num < 0 || rho_den < 1 || rho_num > rho_den)
+        return CALIB_ERR_INVALID;
+    if (static_cast<long long>(H) * nq * nk > (1ll << 31) - 1) return CALIB_ERR_INVALID;
+    if (calib_status s = check_device()) return s;
+    const int rows = H * nq;
+    calib::aggregate_kernel<<<rows_grid(rows), 128, 0, as_stream(stream)>>>(counts, rows, nk, n_inputs, rho_num,
+                                                                             rho_den, mask_out);
+    return launch_status();
+}
+
+calib_status calib_mask_to_csr(const uint8_t* mask, int H, int nq, int nk, int32_t* row_ptr_out,
+                               int16_t* col_idx_out, void* stream) {
+    if (!mask || !row_ptr_out || !col_idx_out) return CALIB_ERR_INVALID;
+    if (H < 1 || nq < 1 || nk < 1 || nk > 32767) return CALIB_ERR_INVALID;
+    if (static_cast<long long>(H) * nq * nk > (1ll << 31) - 1) return CALIB_ERR_INVALID;
+    if (calib_status s = check_device()) return s;
+    const int rows = H * nq;
+    cudaStream_t st = as_stream(stream);
+    calib::csr_count_kernel<<<rows_grid(rows), 128, 0, st>>>(mask, rows, nk, row_ptr_out);
+    calib::csr_scan_kernel<<<1, 1024, 0, st>>>(row_ptr_out, rows);
+    calib::csr_fill_kernel<<<rows_grid(rows), 128, 0, st>>>(mask, rows, nk, row_ptr_out, col_idx_out);
+    return launch_status();
+}
+
+calib_status calib_build_schedule(const int32_t* row_ptr, int H, int nq, int32_t* work_out, void* stream) {
+    if (!row_ptr || !work_out) return CALIB_ERR_INVALID;
+    if (H < 1 || nq < 1 || H > 32767 || nq > 65535) return CALIB_ERR_INVALID;
+    if (calib_status s = check_device()) return s;
+    const int bytes = calib::kSchedBins * 4;
+    if (calib_status s = ensure_smem(reinterpret_cast<const void*>(calib::schedule_kernel), bytes)) return s;
+    calib::schedule_kernel<<<1, 1024, bytes, as_stream(stream)>>>(row_ptr, H * nq, nq, work_out);
+    return launch_status();
+}
+
+int64_t calib_anchor_count(int F, int Hl, int Wl, int n_text, int stride) {
+    if (F < 1 || Hl < 1 || Wl < 1 || n_text < 0 || stride < 1) return -1;
+    const int64_t Ar = (Hl + stride - 1) / stride;
+    return static_cast<int64_t>(F) * Ar * Wl + n_text;
+}
+
+calib_status calib_anchor_rows(int F, int Hl, int Wl, int n_text, int stride, int32_t* rows_out, void* stream) {
+    const int64_t na = calib_anchor_count(F, Hl, Wl, n_text, stride);
+    if (!rows_out || na < 0 || static_cast<int64_t>(F) * Hl * Wl + n_text > (1ll << 31) - 1) return CALIB_ERR_INVALID;
+    if (calib_status s = check_device()) return s;
+    const int Ar = (Hl + stride - 1) / stride;
+    const int n = static_cast<int>(na);
+    calib::anchor_rows_kernel<<<cdiv(n, 256), 256, 0, as_stream(stream)>>>(F, Hl, Wl, n_text, stride, Ar, n,
+                                                                            rows_out);
+    return launch_status();
+}
+
+calib_status sparse_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse_opt, int H, int N,
+                             int D, float scale, const calib_block_list* list, uint32_t flags, void* stream) {
+    return attn_common(q, k, v, o, lse_opt, H, N, D, scale, list, nullptr, 1, 1, N, 0, 1, flags, stream);
+}
+
+calib_status sparse_attn_fwd_repeat(const void* q, const void* k, const void* v, void* o, float* lse_opt, int H,
+                                    int D, int F, int Hl, int Wl, int n_text, int stride,
+                                    const uint8_t* head_repeat, float scale, const calib_block_list* list,
+                                    uint32_t flags, void* stream) {
+    if (!head_repeat || calib_anchor_count(F, Hl, Wl, n_text, stride) < 0 || H < 1 || H > 1024)
+        return CALIB_ERR_INVALID;
+    const long long N = static_cast<long long>(F) * Hl * Wl + n_text;
+    if (N > (1ll << 31) - 1) return CALIB_ERR_INVALID;
+    uint32_t bits[32] = {0};
+    for (int h = 0; h < H; ++h)
+        if (head_repeat[h]) bits[h >> 5] |= 1u << (h & 31);
+    return attn_common(q, k, v, o, lse_opt, H, static_cast<int>(N), D, scale, list, bits, F, Hl, Wl, n_text,
+                       stride, flags, stream);
+}
+
+calib_status calib_selftest_wait_timeout(uint32_t timeout_us, void* stream) {
+    if (calib_status s = check_device()) return s;
+    calib::selftest_wait_kernel<<<1, 32, 0, as_stream(stream)>>>(static_cast<uint64_t>(timeout_us) * 1000ull);
+    if (cudaGetLastError() != cudaSuccess) return CALIB_ERR_CUDA;
+    return calib_device_check(stream);
+}
+
+}  // extern "C"

@@ -1,0 +1,430 @@
+// Block-sparse attention forward for sm_100a: tcgen05 MMAs accumulating in tensor
+// memory, TMA-fed Q/K/V tiles, warp-specialised roles.
+//
+// The method computes attention only on the (query block, key block) tiles its
+// calibrated skip list keeps, densely inside each tile (summaries of "Accelerating
+// Text-to-Video Generation with Calibrated Sparse Attention": [zh] §2.2B, [de] §2B,
+// [fr] §2.C), and for spatial-repetition heads only on anchor rows whose output is
+// broadcast to the other rows of their frame ([zh] §2.2B, [fr] §2.C).
+//
+// One CTA per work item (head h, query block i).  192 threads:
+//   warp 0      TMA producer: Q tile once (or nothing for repeat heads, whose anchor
+//               rows are gathered by the softmax warps), then K_j / V_j for each kept j
+//               through KST / VST-deep rings.
+//   warp 1      TMEM owner (512 columns) and single-thread MMA issuer:
+//               S_t = Q K_j^T  (SS MMA, M=128, N=B, K=D) into S buffer t%2,
+//               O  += P_t V_j  (TS MMA: P from TMEM, V from SMEM, M=128, N=D, K=B).
+//   warps 2..5  softmax + epilogue, one query row per thread (TMEM lane = row):
+//               online max/sum in the log2 domain with lazy rescaling of O, P written
+//               back to TMEM as bf16 over S's columns, final 1/l, bf16 stores.
+// Tensor memory: S0 = cols [0,128), S1 = [128,256), O = [256, 256+D).
+#pragma once
+#include <cuda_bf16.h>
+#include "ptx.cuh"
+
+namespace calib {
+
+constexpr int kAttnThreads = 192;
+constexpr int kTileM = 128;               // query rows per tile (MMA M)
+constexpr float kRescaleLog2 = 8.0f;      // rescale O only when the row max grows by > 2^8
+constexpr uint32_t kTmemCols = 512;
+
+struct AttnParams {
+    const __nv_bfloat16* q;   // [H, N, D] (read directly only for repeat-head gathers)
+    __nv_bfloat16* o;         // [H, N, D], bf16 (or fp32 when out_f32)
+    float* lse;               // [H, N] or nullptr
+    const int32_t* row_ptr;   // [H*nq + 1]
+    const int16_t* col_idx;
+    const int32_t* work;      // [n_items] (h << 16 | i) or nullptr (row order)
+    int H, N, nq, nk;
+    float scale_log2;         // scale * log2(e)
+    // spatial repetition
+    int F, Hl, Wl, n_text, stride, Ar, n_anchor, nq_anchor;
+    uint32_t repeat_bits[32]; // bit h set: head h is a repeat head
+    int out_f32;              // 1: o is fp32 [H, N, D]; 0: bf16
+    uint64_t timeout_ns;
+};
+
+// Token index of anchor `a` (compacted order: latent rows 0, s, 2s, ... of each frame,
+// every column; then text tokens).
+__device__ __forceinline__ int anchor_token(const AttnParams& p, int a) {
+    const int per_frame = p.Ar * p.Wl;
+    const int nva = p.F * per_frame;
+    if (a < nva) {
+        const int f = a / per_frame;
+        const int rem = a - f * per_frame;
+        const int ya = rem / p.Wl;
+        const int x = rem - ya * p.Wl;
+        return (f * p.Hl + ya * p.stride) * p.Wl + x;
+    }
+    return p.F * p.Hl * p.Wl + (a - nva);
+}
+
+// Gather one 128-byte-swizzled Q row (D bf16) from global memory into the tile.
+template <int D>
+__device__ __forceinline__ void gather_q_row(uint8_t* sQ, int r, const __nv_bfloat16* src) {
+#pragma unroll
+    for (int c16 = 0; c16 < D / 8; ++c16) {
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (src) v = __ldg(reinterpret_cast<const uint4*>(src) + c16);
+        const int atom = c16 >> 3, chunk = c16 & 7;
+        uint8_t* dst = sQ + atom * (kTileM * 128) + r * 128 + ((chunk ^ (r & 7)) << 4);
+        *reinterpret_cast<uint4*>(dst) = v;
+    }
+}
+
+// Write one output row (D values already scaled, fp32 in registers, 32 per chunk).
+__device__ __forceinline__ void store_row_chunk(__nv_bfloat16* dst, const uint32_t (&packed)[16]) {
+    uint4* d = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+    for (int v = 0; v < 4; ++v)
+        d[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
+}
+
+template <int D, int BLK, int KST, int VST>
+struct AttnSmem {
+    static constexpr int CH = D / 64;                     // 128-byte chunks per row
+    static constexpr uint32_t Q_BYTES = CH * kTileM * 128;
+    static constexpr uint32_t KV_BYTES = CH * BLK * 128;
+    static constexpr uint32_t OFF_K = Q_BYTES;
+    static constexpr uint32_t OFF_V = OFF_K + KST * KV_BYTES;
+    static constexpr uint32_t OFF_BAR = OFF_V + VST * KV_BYTES;
+    // barrier indices
+    static constexpr int B_Q = 0, B_KF = 1, B_KE = B_KF + KST, B_VF = B_KE + KST,
+                         B_VE = B_VF + VST, B_SF = B_VE + VST, B_PF = B_SF + 2, B_O = B_PF + 2,
+                         B_DRAIN = B_O + 1, NBARS = B_DRAIN + 1;
+    static constexpr uint32_t OFF_MISC = OFF_BAR + NBARS * 8;
+    // + alignment slack; at least 120 KB so that one CTA (holding all 512 TMEM columns)
+    // is resident per SM and no CTA waits in tcgen05.alloc.
+    static constexpr uint32_t RAW = OFF_MISC + 16 + 1024;
+    static constexpr uint32_t BYTES = RAW > 120u * 1024 ? RAW : 120u * 1024;
+};
+
+template <int D, int BLK, int KST, int VST>
+__global__ void __launch_bounds__(kAttnThreads, 1)
+attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
+    using L = AttnSmem<D, BLK, KST, VST>;
+    constexpr int CH = L::CH;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~static_cast<uintptr_t>(1023));
+    uint8_t* sQ = smem;
+    uint8_t* sK = smem + L::OFF_K;
+    uint8_t* sV = smem + L::OFF_V;
+    const uint32_t bar0 = smem_u32(smem + L::OFF_BAR);
+    auto bar = [&](int idx) -> uint32_t { return bar0 + 8u * idx; };
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
+
+    const uint32_t warp = warp_id(), lane = lane_id();
+
+    // ---- work item --------------------------------------------------------------
+    int h, i;
+    if (p.work) {
+        const int item = p.work[blockIdx.x];
+        h = item >> 16;
+        i = item & 0xFFFF;
+    } else {
+        h = blockIdx.x / p.nq;
+        i = blockIdx.x - h * p.nq;
+    }
+    const bool rep = (p.repeat_bits[h >> 5] >> (h & 31)) & 1u;
+    const int Nq = rep ? p.n_anchor : p.N;
+    if (i >= (rep ? p.nq_anchor : p.nq)) return;  // rows past a repeat head's anchor space
+    const int lrow = h * p.nq + i;
+    const int kbeg = p.row_ptr[lrow];
+    const int nkept = p.row_ptr[lrow + 1] - kbeg;
+
+    // ---- setup ------------------------------------------------------------------
+    if (threadIdx.x == 0) {
+        mbar_init(bar(L::B_Q), rep ? 128u : 1u);
+        for (int s = 0; s < KST; ++s) { mbar_init(bar(L::B_KF + s), 1); mbar_init(bar(L::B_KE + s), 1); }
+        for (int s = 0; s < VST; ++s) { mbar_init(bar(L::B_VF + s), 1); mbar_init(bar(L::B_VE + s), 1); }
+        for (int b = 0; b < 2; ++b) { mbar_init(bar(L::B_SF + b), 1); mbar_init(bar(L::B_PF + b), 128); }
+        mbar_init(bar(L::B_O), 1);
+        mbar_init(bar(L::B_DRAIN), 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tm_q);
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_v);
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const WaitCtl ctl{abort_flag, p.timeout_ns};
+
+    // bookkeeping for the abort drain (producer only)
+    int armed_q = 0, armed_k[KST], armed_v[VST];
+#pragma unroll
+    for (int s = 0; s < KST; ++s) armed_k[s] = 0;
+#pragma unroll
+    for (int s = 0; s < VST; ++s) armed_v[s] = 0;
+
+    if (warp == 0) {
+        // ===================== TMA producer =====================
+        if (lane == 0 && nkept > 0) {
+            if (!rep) {
+                mbar_arrive_expect_tx(bar(L::B_Q), L::Q_BYTES);
+                for (int c = 0; c < CH; ++c)
+                    tma_load_3d(smem_u32(sQ + c * kTileM * 128), &tm_q, bar(L::B_Q), c * 64, i * BLK, h);
+                armed_q = 1;
+            }
+            auto issue_k = [&](int t) -> bool {
+                const int s = t % KST;
+                if (!mbar_wait(bar(L::B_KE + s), ((t / KST) & 1) ^ 1, ctl)) return false;
+                const int j = p.col_idx[kbeg + t];
+                mbar_arrive_expect_tx(bar(L::B_KF + s), L::KV_BYTES);
+                for (int c = 0; c < CH; ++c)
+                    tma_load_3d(smem_u32(sK + s * L::KV_BYTES + c * BLK * 128), &tm_k, bar(L::B_KF + s),
+                                c * 64, j * BLK, h);
+                ++armed_k[s];
+                return true;
+            };
+            auto issue_v = [&](int t) -> bool {
+                const int s = t % VST;
+                if (!mbar_wait(bar(L::B_VE + s), ((t / VST) & 1) ^ 1, ctl)) return false;
+                const int j = p.col_idx[kbeg + t];
+                mbar_arrive_expect_tx(bar(L::B_VF + s), L::KV_BYTES);
+                for (int c = 0; c < CH; ++c)
+                    tma_load_3d(smem_u32(sV + s * L::KV_BYTES + c * BLK * 128), &tm_v, bar(L::B_VF + s),
+                                c * 64, j * BLK, h);
+                ++armed_v[s];
+                return true;
+            };
+            // K runs ahead of V: the MMA order is QK_0, QK_1, PV_0, QK_2, PV_1, ...
+            bool ok = issue_k(0);
+            for (int t = 0; ok && t < nkept; ++t) {
+                if (t + 1 < nkept) ok = issue_k(t + 1);
+                if (ok) ok = issue_v(t);
+            }
+        }
+    } else if (warp == 1) {
+        // ===================== MMA issuer =====================
+        if (lane == 0 && nkept > 0) {
+            constexpr uint32_t idesc_qk = idesc_bf16_f32(kTileM, BLK, false, false);
+            constexpr uint32_t idesc_pv = idesc_bf16_f32(kTileM, D, false, true);
+            const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV);
+            bool ok = mbar_wait(bar(L::B_Q), 0, ctl);
+            tc_fence_after();
+            auto issue_qk = [&](int t) -> bool {
+                const int s = t % KST;
+                if (!mbar_wait(bar(L::B_KF + s), (t / KST) & 1, ctl)) return false;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem + (t & 1) * 128;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t inner = (kk & 3) * 32;   // K step of 16 bf16 inside a 128-B atom
+                    const uint64_t ad = smem_desc_sw128(sQa + (kk >> 2) * kTileM * 128 + inner, 16, 1024);
+                    const uint64_t bd =
+                        smem_desc_sw128(sKa + s * L::KV_BYTES + (kk >> 2) * BLK * 128 + inner, 16, 1024);
+                    umma_ss(d_tmem, ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
+                }
+                umma_commit(bar(L::B_SF + (t & 1)));
+                umma_commit(bar(L::B_KE + s));
+                return true;
+            };
+            if (ok) ok = issue_qk(0);
+            for (int t = 0; ok && t < nkept; ++t) {
+                if (t + 1 < nkept) {
+                    // S buffer (t+1)&1 last held P_{t-1}: PV_{t-1} must be complete.
+                    if (t >= 1) ok = mbar_wait(bar(L::B_O), (t - 1) & 1, ctl);
+                    if (ok) ok = issue_qk(t + 1);
+                    if (!ok) break;
+                }
+                const int sv = t % VST;
+                ok = mbar_wait(bar(L::B_PF + (t & 1)), (t >> 1) & 1, ctl);
+                if (ok) ok = mbar_wait(bar(L::B_VF + sv), (t / VST) & 1, ctl);
+                if (!ok) break;
+                tc_fence_after();
+                const uint32_t a_tmem = tmem + (t & 1) * 128;
+#pragma unroll
+                for (int kk = 0; kk < BLK / 16; ++kk) {
+                    const uint64_t bd =
+                        smem_desc_sw128(sVa + sv * L::KV_BYTES + kk * 16 * 128, BLK * 128, 1024);
+                    umma_ts(tmem + 256, a_tmem + kk * 8, bd, idesc_pv, (t > 0 || kk > 0) ? 1u : 0u);
+                }
+                umma_commit(bar(L::B_O));
+                umma_commit(bar(L::B_VE + sv));
+            }
+        }
+    } else {
+        // ===================== softmax + epilogue (warps 2..5) =====================
+        const uint32_t q4 = warp & 3;
+        const int r = static_cast<int>(q4 * 32 + lane);   // tile row == TMEM lane
+        const uint32_t lane_base = (q4 * 32) << 16;
+        if (rep && nkept > 0) {
+            const int a = i * BLK + r;
+            const __nv_bfloat16* src =
+                (a < Nq) ? p.q + (static_cast<size_t>(h) * p.N + anchor_token(p, a)) * D : nullptr;
+            gather_q_row<D>(sQ, r, src);
+            fence_proxy_async_smem();
+            mbar_arrive(bar(L::B_Q));
+        }
+        float m_run = -INFINITY, l_run = 0.f, lq_run = 0.f;
+        bool ok = true;
+        for (int t = 0; t < nkept; ++t) {
+            const int j = p.col_idx[kbeg + t];
+            const int valid = min(BLK, p.N - j * BLK);
+            ok = mbar_wait_warp(bar(L::B_SF + (t & 1)), (t >> 1) & 1, ctl);
+            if (!ok) break;
+            tc_fence_after();
+            float s[BLK];
+            {
+                uint32_t raw[32];
+#pragma unroll
+                for (int c = 0; c < BLK / 32; ++c) {
+                    tmem_ld32(tmem + lane_base + (t & 1) * 128 + c * 32, raw);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) s[c * 32 + e] = __uint_as_float(raw[e]);
+                }
+            }
+            float mt = -INFINITY;
+#pragma unroll
+            for (int c = 0; c < BLK; ++c)
+                if (c < valid) mt = fmaxf(mt, s[c]);
+            const float mt2 = mt * p.scale_log2;
+            const bool upd = mt2 > m_run + kRescaleLog2;
+            const float m_new = upd ? mt2 : m_run;
+            const float alpha = upd ? ex2_approx(m_run - m_new) : 1.f;
+            // P enters the PV MMA as bf16; O is normalised by the sum of those rounded
+            // weights (lq), so O stays an exact convex combination of the weights used.
+            // The unrounded sum (l) gives the LSE output.
+            float sum = 0.f, sumq = 0.f;
+            uint32_t pk[BLK / 2];
+#pragma unroll
+            for (int c = 0; c < BLK; c += 2) {
+                const float p0 = (c < valid) ? ex2_approx(fmaf(s[c], p.scale_log2, -m_new)) : 0.f;
+                const float p1 = (c + 1 < valid) ? ex2_approx(fmaf(s[c + 1], p.scale_log2, -m_new)) : 0.f;
+                sum += p0 + p1;
+                const uint32_t w = pack_bf16x2(p0, p1);
+                sumq += __uint_as_float(w << 16) + __uint_as_float(w & 0xFFFF0000u);
+                pk[c / 2] = w;
+            }
+            l_run = l_run * alpha + sum;
+            lq_run = lq_run * alpha + sumq;
+            m_run = m_new;
+#pragma unroll
+            for (int c = 0; c < BLK / 32; ++c)
+                tmem_st16(tmem + lane_base + (t & 1) * 128 + c * 16, pk + c * 16);
+            if (__any_sync(0xffffffffu, upd && t > 0)) {
+                // O accumulated through PV_{t-1}: wait for it, then rescale rows in place.
+                ok = mbar_wait_warp(bar(L::B_O), (t - 1) & 1, ctl);
+                if (!ok) break;
+                tc_fence_after();
+                const float a_row = (upd && t > 0) ? alpha : 1.f;
+                uint32_t raw[32];
+#pragma unroll
+                for (int c = 0; c < D / 32; ++c) {
+                    tmem_ld32(tmem + lane_base + 256 + c * 32, raw);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) raw[e] = __float_as_uint(__uint_as_float(raw[e]) * a_row);
+                    tmem_st32(tmem + lane_base + 256 + c * 32, raw);
+                }
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(bar(L::B_PF + (t & 1)));
+        }
+        // ---- epilogue ----
+        if (__all_sync(0xffffffffu, ok && !*abort_flag)) {
+            const bool row_ok = r < BLK && (i * BLK + r) < Nq;
+            if (nkept > 0) ok = mbar_wait_warp(bar(L::B_O), (nkept - 1) & 1, ctl);
+            if (ok) {
+                tc_fence_after();
+                const float inv_l = nkept > 0 ? 1.f / lq_run : 0.f;
+                const float lse_val = nkept > 0 ? (m_run + lg2_approx(l_run)) * 0.69314718055994530942f : -INFINITY;
+                // destination rows: the row itself, or every token an anchor stands for
+                int tok0 = 0, ncopy = 0, copy_stride = 0;
+                if (row_ok) {
+                    const int a = i * BLK + r;
+                    if (!rep) {
+                        tok0 = a; ncopy = 1;
+                    } else {
+                        const int nva = p.F * p.Ar * p.Wl;
+                        if (a < nva) {
+                            tok0 = anchor_token(p, a);
+                            const int ya = (a / p.Wl) % p.Ar;
+                            ncopy = min(p.stride, p.Hl - ya * p.stride);
+                            copy_stride = p.Wl;
+                        } else {
+                            tok0 = anchor_token(p, a); ncopy = 1;
+                        }
+                    }
+                }
+                uint32_t raw[32];
+#pragma unroll
+                for (int c = 0; c < D / 32; ++c) {
+                    if (nkept > 0) {
+                        tmem_ld32(tmem + lane_base + 256 + c * 32, raw);
+                        tmem_wait_ld();
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) raw[e] = 0u;
+                    }
+                    if (p.out_f32) {
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) raw[e] = __float_as_uint(__uint_as_float(raw[e]) * inv_l);
+                        for (int cp = 0; cp < ncopy; ++cp) {
+                            const size_t tok = static_cast<size_t>(tok0 + cp * copy_stride);
+                            uint4* d = reinterpret_cast<uint4*>(reinterpret_cast<float*>(p.o) +
+                                                                (static_cast<size_t>(h) * p.N + tok) * D + c * 32);
+#pragma unroll
+                            for (int v4 = 0; v4 < 8; ++v4)
+                                d[v4] = make_uint4(raw[4 * v4], raw[4 * v4 + 1], raw[4 * v4 + 2], raw[4 * v4 + 3]);
+                        }
+                    } else {
+                        uint32_t packed[16];
+#pragma unroll
+                        for (int e = 0; e < 16; ++e)
+                            packed[e] = pack_bf16x2(__uint_as_float(raw[2 * e]) * inv_l,
+                                                    __uint_as_float(raw[2 * e + 1]) * inv_l);
+                        for (int cp = 0; cp < ncopy; ++cp) {
+                            const size_t tok = static_cast<size_t>(tok0 + cp * copy_stride);
+                            store_row_chunk(p.o + (static_cast<size_t>(h) * p.N + tok) * D + c * 32, packed);
+                        }
+                    }
+                }
+                if (p.lse)
+                    for (int cp = 0; cp < ncopy; ++cp)
+                        p.lse[static_cast<size_t>(h) * p.N + tok0 + cp * copy_stride] = lse_val;
+            }
+        }
+    }
+
+    // ---- teardown (also the abort drain) ----------------------------------------
+    // After this barrier no role waits any more, so every thread reads the same flag.
+    __syncthreads();
+    if (*abort_flag) {
+        constexpr uint64_t kDrainNs = 1000000000ull;
+        if (warp == 0 && lane == 0) {
+            if (armed_q) mbar_wait_drain(bar(L::B_Q), 0, kDrainNs);
+            for (int s = 0; s < KST; ++s)
+                if (armed_k[s]) mbar_wait_drain(bar(L::B_KF + s), (armed_k[s] - 1) & 1, kDrainNs);
+            for (int s = 0; s < VST; ++s)
+                if (armed_v[s]) mbar_wait_drain(bar(L::B_VF + s), (armed_v[s] - 1) & 1, kDrainNs);
+        }
+        if (warp == 1 && lane == 0) {
+            umma_commit(bar(L::B_DRAIN));
+            mbar_wait_drain(bar(L::B_DRAIN), 0, kDrainNs);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+}  // namespace calib

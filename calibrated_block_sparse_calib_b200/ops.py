@@ -1,0 +1,291 @@
+"""ctypes binding of libcalibatt.so (see include/calibatt.h for the semantics).
+
+Argument marshalling only: every function checks dtypes, shapes and devices, allocates
+outputs with torch (device memory), and calls the C ABI on torch's current CUDA stream.
+All arithmetic runs in the library's sm_100a kernels.  There is no fallback: a missing
+library or a non-CUDA tensor raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from dataclasses import dataclass
+from typing import Optional, Sequence
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libcalibatt.so")
+
+CALIB_OK, CALIB_ERR_INVALID, CALIB_ERR_UNSUPPORTED, CALIB_ERR_CUDA, CALIB_ERR_TIMEOUT = range(5)
+CALIB_ATTN_OUT_F32 = 1
+
+
+class CalibError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn} failed: {status_string(status)} ({status})")
+
+
+class _BlockListC(ctypes.Structure):
+    _fields_ = [("H", ctypes.c_int32), ("nq", ctypes.c_int32), ("nk", ctypes.c_int32),
+                ("block", ctypes.c_int32), ("row_ptr", ctypes.c_void_p), ("col_idx", ctypes.c_void_p),
+                ("work", ctypes.c_void_p), ("n_work", ctypes.c_int32)]
+
+
+_lib = None
+_P, _I, _F, _D, _U32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_double, ctypes.c_uint32
+_SIGS = {
+    "calib_status_string": ([ctypes.c_int], ctypes.c_char_p),
+    "calib_device_check": ([_P], ctypes.c_int),
+    "calib_block_energy": ([_P, _P, _P, _I, _I, _I, _I, _F, _P, _I, _P, _I, _P], ctypes.c_int),
+    "calib_select_mask": ([_P, _I, _I, _I, _D, _P, _P, _P, _P], ctypes.c_int),
+    "calib_aggregate_masks": ([_P, _I, _I, _I, _I, _I, _I, _P, _P], ctypes.c_int),
+    "calib_mask_to_csr": ([_P, _I, _I, _I, _P, _P, _P], ctypes.c_int),
+    "calib_build_schedule": ([_P, _I, _I, _P, _P], ctypes.c_int),
+    "calib_anchor_count": ([_I, _I, _I, _I, _I], ctypes.c_int64),
+    "calib_anchor_rows": ([_I, _I, _I, _I, _I, _P, _P], ctypes.c_int),
+    "sparse_attn_fwd": ([_P, _P, _P, _P, _P, _I, _I, _I, _F, ctypes.POINTER(_BlockListC), _U32, _P],
+                        ctypes.c_int),
+    "sparse_attn_fwd_repeat": ([_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _F,
+                                ctypes.POINTER(_BlockListC), _U32, _P], ctypes.c_int),
+    "calib_selftest_wait_timeout": ([_U32, _P], ctypes.c_int),
+}
+
+
+def lib():
+    """Load libcalibatt.so (built in-tree); raises if it is missing."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: run `python -m calibrated_block_sparse_calib_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (args, res) in _SIGS.items():
+            f = getattr(L, name)
+            f.argtypes = args
+            f.restype = res
+        _lib = L
+    return _lib
+
+
+def status_string(s: int) -> str:
+    return lib().calib_status_string(int(s)).decode()
+
+
+def _check(fn: str, s: int):
+    if s != CALIB_OK:
+        raise CalibError(fn, s)
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _need(t: torch.Tensor, name: str, dtype: torch.dtype, shape=None):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def device_check():
+    """Synchronise the current stream and raise if a kernel recorded an error."""
+    _check("calib_device_check", lib().calib_device_check(_stream()))
+
+
+def selftest_wait_timeout(timeout_us: int = 1000) -> int:
+    """Run the bounded-wait self-test; returns the status (CALIB_ERR_TIMEOUT expected)."""
+    return lib().calib_selftest_wait_timeout(int(timeout_us), _stream())
+
+
+def nblocks(n: int, block: int) -> int:
+    return (n + block - 1) // block
+
+
+# ----------------------------------------------------------------------------------
+# calibration
+# ----------------------------------------------------------------------------------
+
+def block_energy(q: torch.Tensor, k: torch.Tensor, block: int, scale: Optional[float] = None,
+                 lse: Optional[torch.Tensor] = None, q_rows: Optional[torch.Tensor] = None,
+                 out: Optional[torch.Tensor] = None, accumulate: bool = False) -> torch.Tensor:
+    """fp32 block energies [H, ceil(Nq/B), ceil(N/B)] of softmax(scale q k^T)."""
+    H, N, D = k.shape
+    _need(q, "q", torch.bfloat16, (H, N, D))
+    _need(k, "k", torch.bfloat16)
+    Nq = N
+    if q_rows is not None:
+        _need(q_rows, "q_rows", torch.int32)
+        Nq = q_rows.numel()
+    if lse is not None:
+        _need(lse, "lse", torch.float32, (H, Nq))
+    shape = (H, nblocks(Nq, block), nblocks(N, block))
+    if out is None:
+        out = (torch.zeros if accumulate else torch.empty)(shape, dtype=torch.float32, device=q.device)
+    _need(out, "out", torch.float32, shape)
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    _check("calib_block_energy", lib().calib_block_energy(
+        _ptr(q), _ptr(k), _ptr(lse), H, N, D, block, scale, _ptr(q_rows), Nq if q_rows is not None else 0,
+        _ptr(out), 1 if accumulate else 0, _stream()))
+    return out
+
+
+def select_mask(energy: torch.Tensor, tau: float, force_keep: Optional[torch.Tensor] = None,
+                out: Optional[torch.Tensor] = None, count_accum: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """uint8 keep mask [H, nq, nk] of the minimal tau-energy selection."""
+    _need(energy, "energy", torch.float32)
+    H, nq, nk = energy.shape
+    if force_keep is not None:
+        _need(force_keep, "force_keep", torch.uint8, energy.shape)
+    if out is None:
+        out = torch.empty(energy.shape, dtype=torch.uint8, device=energy.device)
+    _need(out, "out", torch.uint8, energy.shape)
+    if count_accum is not None:
+        _need(count_accum, "count_accum", torch.int32, energy.shape)
+    _check("calib_select_mask", lib().calib_select_mask(
+        _ptr(energy), H, nq, nk, float(tau), _ptr(force_keep), _ptr(out), _ptr(count_accum), _stream()))
+    return out
+
+
+def aggregate_masks(counts: torch.Tensor, n_inputs: int, rho: Sequence[int] = (1, 2),
+                    out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """uint8 mask of blocks kept with frequency strictly above rho = rho[0]/rho[1]."""
+    _need(counts, "counts", torch.int32)
+    H, nq, nk = counts.shape
+    if out is None:
+        out = torch.empty(counts.shape, dtype=torch.uint8, device=counts.device)
+    _need(out, "out", torch.uint8, counts.shape)
+    _check("calib_aggregate_masks", lib().calib_aggregate_masks(
+        _ptr(counts), H, nq, nk, int(n_inputs), int(rho[0]), int(rho[1]), _ptr(out), _stream()))
+    return out
+
+
+def mask_to_csr(mask: torch.Tensor):
+    """(row_ptr int32 [H*nq+1], col_idx int16 [H*nq*nk] capacity) skip list of a mask."""
+    _need(mask, "mask", torch.uint8)
+    H, nq, nk = mask.shape
+    row_ptr = torch.empty(H * nq + 1, dtype=torch.int32, device=mask.device)
+    col_idx = torch.empty(max(1, H * nq * nk), dtype=torch.int16, device=mask.device)
+    _check("calib_mask_to_csr", lib().calib_mask_to_csr(
+        _ptr(mask), H, nq, nk, _ptr(row_ptr), _ptr(col_idx), _stream()))
+    return row_ptr, col_idx
+
+
+def build_schedule(row_ptr: torch.Tensor, H: int, nq: int) -> torch.Tensor:
+    """int32 work list (h << 16 | i), kept count descending, ties by (h, i)."""
+    _need(row_ptr, "row_ptr", torch.int32, (H * nq + 1,))
+    work = torch.empty(H * nq, dtype=torch.int32, device=row_ptr.device)
+    _check("calib_build_schedule", lib().calib_build_schedule(_ptr(row_ptr), H, nq, _ptr(work), _stream()))
+    return work
+
+
+def anchor_count(F: int, Hl: int, Wl: int, n_text: int, stride: int) -> int:
+    n = lib().calib_anchor_count(F, Hl, Wl, n_text, stride)
+    if n < 0:
+        raise ValueError("invalid anchor geometry")
+    return int(n)
+
+
+def anchor_rows(F: int, Hl: int, Wl: int, n_text: int, stride: int, device="cuda") -> torch.Tensor:
+    """int32 token indices of the anchor rows (compacted order)."""
+    rows = torch.empty(anchor_count(F, Hl, Wl, n_text, stride), dtype=torch.int32, device=device)
+    _check("calib_anchor_rows", lib().calib_anchor_rows(F, Hl, Wl, n_text, stride, _ptr(rows), _stream()))
+    return rows
+
+
+# ----------------------------------------------------------------------------------
+# inference
+# ----------------------------------------------------------------------------------
+
+@dataclass
+class BlockList:
+    """Device-resident skip list of one (timestep, layer) slice (see calib_block_list)."""
+    H: int
+    nq: int
+    nk: int
+    block: int
+    row_ptr: torch.Tensor
+    col_idx: torch.Tensor
+    work: Optional[torch.Tensor] = None
+
+    def c_struct(self) -> _BlockListC:
+        _need(self.row_ptr, "row_ptr", torch.int32, (self.H * self.nq + 1,))
+        _need(self.col_idx, "col_idx", torch.int16)
+        if self.work is not None:
+            _need(self.work, "work", torch.int32)
+        return _BlockListC(self.H, self.nq, self.nk, self.block, self.row_ptr.data_ptr(),
+                           self.col_idx.data_ptr(), 0 if self.work is None else self.work.data_ptr(),
+                           0 if self.work is None else self.work.numel())
+
+    @staticmethod
+    def from_mask(mask: torch.Tensor, block: int, schedule: bool = True) -> "BlockList":
+        """Skip list (and longest-first schedule) of a uint8 [H, nq, nk] device mask."""
+        H, nq, nk = mask.shape
+        rp, ci = mask_to_csr(mask)
+        work = build_schedule(rp, H, nq) if schedule else None
+        return BlockList(H, nq, nk, block, rp, ci, work)
+
+
+def _out(q, out, out_dtype):
+    H, N, D = q.shape
+    if out is None:
+        out = torch.empty((H, N, D), dtype=out_dtype, device=q.device)
+    if out.dtype not in (torch.bfloat16, torch.float32):
+        raise TypeError("out must be bf16 or fp32")
+    _need(out, "out", out.dtype, (H, N, D))
+    return out, (CALIB_ATTN_OUT_F32 if out.dtype == torch.float32 else 0)
+
+
+def sparse_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, blist: BlockList,
+                    scale: Optional[float] = None, out: Optional[torch.Tensor] = None,
+                    lse: Optional[torch.Tensor] = None, return_lse: bool = False,
+                    out_dtype: torch.dtype = torch.bfloat16):
+    """Block-sparse attention: O [H, N, D] in bf16 (or fp32 via out_dtype / an fp32 `out`),
+    and the fp32 LSE [H, N] if requested."""
+    H, N, D = q.shape
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n, torch.bfloat16, (H, N, D))
+    out, flags = _out(q, out, out_dtype)
+    if return_lse and lse is None:
+        lse = torch.empty(H, N, dtype=torch.float32, device=q.device)
+    if lse is not None:
+        _need(lse, "lse", torch.float32, (H, N))
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    cs = blist.c_struct()
+    _check("sparse_attn_fwd", lib().sparse_attn_fwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), H, N, D, scale, ctypes.byref(cs), flags, _stream()))
+    return (out, lse) if (return_lse or lse is not None) else out
+
+
+def sparse_attn_fwd_repeat(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, blist: BlockList,
+                           head_repeat: Sequence[bool], F: int, Hl: int, Wl: int, n_text: int, stride: int,
+                           scale: Optional[float] = None, out: Optional[torch.Tensor] = None,
+                           lse: Optional[torch.Tensor] = None, return_lse: bool = False,
+                           out_dtype: torch.dtype = torch.bfloat16):
+    """Block-sparse attention with spatial repetition on the flagged heads."""
+    H, N, D = q.shape
+    if N != F * Hl * Wl + n_text:
+        raise ValueError("N must equal F*Hl*Wl + n_text")
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n, torch.bfloat16, (H, N, D))
+    out, oflags = _out(q, out, out_dtype)
+    if return_lse and lse is None:
+        lse = torch.empty(H, N, dtype=torch.float32, device=q.device)
+    if lse is not None:
+        _need(lse, "lse", torch.float32, (H, N))
+    flags = (ctypes.c_uint8 * H)(*[1 if bool(x) else 0 for x in head_repeat])
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    cs = blist.c_struct()
+    _check("sparse_attn_fwd_repeat", lib().sparse_attn_fwd_repeat(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), H, D, F, Hl, Wl, n_text, stride,
+        ctypes.cast(flags, ctypes.c_void_p), scale, ctypes.byref(cs), oflags, _stream()))
+    return (out, lse) if (return_lse or lse is not None) else out

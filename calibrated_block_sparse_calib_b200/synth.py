@@ -104,10 +104,11 @@ def token_coords(shape: VideoShape):
 
 
 def make_qkv(wl: Workload, input_idx: int = 0, device="cpu", pos_scale: Optional[float] = None,
-             dtype=torch.bfloat16, heads: Optional[int] = None):
+             dtype=torch.bfloat16, heads: Optional[int] = None, seed: Optional[int] = None):
     """Seeded Q, K, V of shape [H, N, D] in bf16 on `device`.
 
-    The generator is torch.Generator(device) seeded 1000*cfg + input_idx; draw order
+    The generator is torch.Generator(device) seeded 1000*cfg + input_idx (or
+    seed + input_idx for ad-hoc shapes); draw order
     Omega, beta, then per head U_h, Z_q, Z_k, Z_v.  The same seed on the same device
     type gives the same tensors on every call.
     """
@@ -116,7 +117,7 @@ def make_qkv(wl: Workload, input_idx: int = 0, device="cpu", pos_scale: Optional
     s = wl.pos_scale if pos_scale is None else pos_scale
     dev = torch.device(device)
     g = torch.Generator(device=dev)
-    g.manual_seed(1000 * WORKLOAD_INDEX[wl.name] + input_idx)
+    g.manual_seed((1000 * WORKLOAD_INDEX[wl.name] if seed is None else seed) + input_idx)
     r = wl.rank
     omega = torch.randn(r, 3, generator=g, device=dev, dtype=torch.float32)
     beta = torch.rand(r, generator=g, device=dev, dtype=torch.float32) * (2 * math.pi)

@@ -1,0 +1,188 @@
+/*
+ * calibatt.h -- C ABI of libcalibatt.so: calibrated block-sparse attention on one
+ * NVIDIA B200 (sm_100a).
+ *
+ * The method is the one described in the summaries of "Accelerating Text-to-Video
+ * Generation with Calibrated Sparse Attention" (gist.science pages in Chinese, German,
+ * Portuguese and French): offline, energy-based block selection aggregated over
+ * calibration inputs into a static per-(timestep, layer, head) block mask and skip list;
+ * at inference, attention that computes only the kept (query block, key block) tiles,
+ * plus a spatial-repetition mode that computes anchor rows and broadcasts their output.
+ * Section citations below use the tags [zh] technical summary §2.1/§2.2A/§2.2B,
+ * [de] "Technische Zusammenfassung" §2A/§2B, [pt] "Resumo técnico" §2A/§2B,
+ * [fr] "Résumé technique" §2.A/§2.B/§2.C, and [AdaSpa] for the page "Training-free and
+ * Adaptive Sparse Attention for Efficient Long Video Generation" §2.
+ *
+ * Conventions shared by every call:
+ *  - Every pointer is a DEVICE pointer unless its comment says "host".  The caller
+ *    allocates and owns all memory; the library allocates nothing and keeps no state
+ *    other than one device-side status word per device (see calib_device_check).
+ *  - `stream` is a cudaStream_t passed as void*; NULL means the legacy default stream.
+ *    Calls are asynchronous: they validate arguments on the host, enqueue kernels on
+ *    `stream` and return.  No call synchronises, except calib_device_check.
+ *  - Q, K, V, O are bf16, shape [H, N, D] for batch 1, contiguous with D innermost
+ *    (row n of head h starts at element (h*N + n)*D).  Pointers must be 16-byte aligned.
+ *  - Blocks: block size B in {64, 128}; block i covers rows [iB, min((i+1)B, len)).
+ *    nq = ceil(Nq / B) query blocks, nk = ceil(N / B) key blocks; the last one may be
+ *    ragged.
+ *  - Masks are uint8 [H, nq, nk] (0 = skip, 1 = keep), row (h, i) at (h*nq + i)*nk.
+ *  - Errors: CALIB_ERR_INVALID for a null or misaligned pointer or an out-of-range size,
+ *    CALIB_ERR_UNSUPPORTED for a size or device this build does not handle (D not in
+ *    {64,128}, nk > 1024 in selection, a device other than sm_100), CALIB_ERR_CUDA for
+ *    a failed launch.  On an error nothing is enqueued.  Device-side waits are bounded:
+ *    a kernel that gives up records CALIB_ERR_TIMEOUT in the status word and returns.
+ */
+#ifndef CALIBATT_H
+#define CALIBATT_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Flags of the attention calls. */
+#define CALIB_ATTN_OUT_F32 1u   /* o is fp32 [H, N, D] instead of bf16 */
+
+typedef enum calib_status {
+    CALIB_OK = 0,
+    CALIB_ERR_INVALID = 1,
+    CALIB_ERR_UNSUPPORTED = 2,
+    CALIB_ERR_CUDA = 3,
+    CALIB_ERR_TIMEOUT = 4
+} calib_status;
+
+/* Skip list of one (timestep, layer) slice: the kept key blocks of every (head, query
+ * block) row in CSR form ([zh] §2.2B, [pt] §2A.5, [fr] §2.C: the mask is converted into
+ * the list of block intervals to compute, precomputed before inference).
+ * Row r = h*nq + i holds col_idx[row_ptr[r] .. row_ptr[r+1]) in ascending order.
+ * `work` (optional) is the order in which rows are processed: entries h << 16 | i,
+ * longest rows first (calib_build_schedule); NULL processes rows in index order.
+ * All arrays are device memory owned by the caller. */
+typedef struct calib_block_list {
+    int32_t H, nq, nk, block;
+    const int32_t* row_ptr;   /* [H*nq + 1], row_ptr[0] = 0, non-decreasing */
+    const int16_t* col_idx;   /* [row_ptr[H*nq]], each in [0, nk) */
+    const int32_t* work;      /* [n_work] or NULL */
+    int32_t n_work;           /* entries in `work` (ignored when work == NULL) */
+} calib_block_list;
+
+/* Human-readable name of a status code (static storage). */
+const char* calib_status_string(calib_status s);
+
+/* Synchronises `stream`, then reads and clears the status word of the current device.
+ * Returns CALIB_ERR_TIMEOUT if any kernel since the last check gave up on a bounded
+ * wait, CALIB_ERR_INVALID if a selection kernel met a negative or non-finite energy
+ * (treated as 0), CALIB_ERR_CUDA on a CUDA error, else CALIB_OK. */
+calib_status calib_device_check(void* stream);
+
+/* Row log-sum-exp and block energies, fused ([zh] §2.2A, [de] §2A.1, [fr] §2.B.1: split
+ * the post-softmax attention matrix P into B x B blocks and sum each block):
+ *   energy[h, i, j] (+)= sum_{r in I_i, c in J_j} exp(scale * q_r.k_c - LSE_r)
+ * where LSE_r = log sum_c exp(scale * q_r.k_c) over all N keys.
+ *   q, k     : bf16 [H, N, D].
+ *   lse      : NULL, or a cached natural-log LSE fp32 [H, Nq] (e.g. sparse_attn_fwd's
+ *              lse_opt of a dense call; [AdaSpa] §2 caches the LSE this way).  NULL makes
+ *              the kernel compute it first, in registers, with a second pass over K.
+ *   q_rows   : NULL (query rows are the N tokens) or int32 [n_q] token indices in
+ *              compacted order -- the anchor rows of a spatial-repetition head
+ *              (calib_anchor_rows); then Nq = n_q and blocks are over that sequence.
+ *   energy   : fp32 [H, ceil(Nq/B), ceil(N/B)].  accumulate != 0 adds to it (for the
+ *              energy-sum aggregation over inputs); 0 overwrites.
+ * P is never written to memory. */
+calib_status calib_block_energy(const void* q, const void* k, const float* lse,
+                                int H, int N, int D, int block, float scale,
+                                const int32_t* q_rows, int n_q,
+                                float* energy, int accumulate, void* stream);
+
+/* Minimal tau-energy selection ([fr] §2.B.1: per query block, the fewest key blocks whose
+ * cumulative energy reaches the threshold; [zh] §2.2A, [de] §2A.2), one warp per row:
+ *   energy     : fp32 [H, nq, nk], finite and >= 0.
+ *   tau        : in (0, 1]; the per-timestep threshold eps(t).
+ *   force_keep : NULL or uint8 [H, nq, nk]; forced blocks are kept first and count
+ *                toward the threshold (text rows/columns of joint attention).
+ *   mask_out   : uint8 [H, nq, nk].
+ *   count_accum: NULL or int32 [H, nq, nk]; when given, mask_out is also added to it
+ *                (the per-input masks of the cross-prompt vote).
+ * Arithmetic is exact integer: each row is scaled by a power of two into integers
+ * q_j < 2^53 (rounded half-even), T = max(1, ceil(tau * sum q)) with one IEEE double
+ * multiply, and the kept set is forced blocks plus the largest q_j (lower key index
+ * first on ties) until the sum reaches T.  A row whose energies are all 0 keeps block
+ * i (block 0 if i >= nk) and its forced blocks.  nk <= 1024. */
+calib_status calib_select_mask(const float* energy, int H, int nq, int nk, double tau,
+                               const uint8_t* force_keep, uint8_t* mask_out,
+                               int32_t* count_accum, void* stream);
+
+/* Cross-input vote ([zh] §2.2A, [de] §2A.3, [fr] §2.B.2): keep (h, i, j) iff
+ * counts[h,i,j] * rho_den > rho_num * n_inputs (frequency strictly above rho =
+ * rho_num/rho_den).  A row left empty keeps its most frequent block (lowest index on
+ * ties).  counts: int32 [H, nq, nk] in [0, n_inputs]; mask_out: uint8 [H, nq, nk]. */
+calib_status calib_aggregate_masks(const int32_t* counts, int H, int nq, int nk,
+                                   int n_inputs, int rho_num, int rho_den,
+                                   uint8_t* mask_out, void* stream);
+
+/* Skip list from a mask: row_ptr_out int32 [H*nq + 1], col_idx_out int16 with capacity
+ * for every kept block (H*nq*nk always suffices).  nk <= 32767. */
+calib_status calib_mask_to_csr(const uint8_t* mask, int H, int nq, int nk,
+                               int32_t* row_ptr_out, int16_t* col_idx_out, void* stream);
+
+/* Load-balancing order ([AdaSpa] §2 balances kernel load across heads of different
+ * sparsity): work_out int32 [H*nq] = every row h << 16 | i, kept count descending, ties
+ * by (h, i) ascending.  H, nq < 65536. */
+calib_status calib_build_schedule(const int32_t* row_ptr, int H, int nq,
+                                  int32_t* work_out, void* stream);
+
+/* Number of anchor tokens of a spatial-repetition head: F * ceil(Hl/stride) * Wl +
+ * n_text (host computation, no device work).  Returns -1 for invalid sizes. */
+int64_t calib_anchor_count(int F, int Hl, int Wl, int n_text, int stride);
+
+/* Anchor token indices in compacted order ([zh] §2.1, [fr] §2.A.4, §2.C: only anchor rows
+ * of a frame are computed and broadcast to the other rows of the frame): latent rows
+ * y = 0, s, 2s, ... of each frame, all columns, then the text tokens.
+ * rows_out: int32 [calib_anchor_count(...)]. */
+calib_status calib_anchor_rows(int F, int Hl, int Wl, int n_text, int stride,
+                               int32_t* rows_out, void* stream);
+
+/* Block-sparse attention forward ([zh] §2.2B, [de] §2B, [pt] §2B, [fr] §2.C: compute the
+ * kept blocks densely, skip the rest):
+ *   O_r = sum_{c in K(i)} softmax_{c in K(i)}(scale * q_r.k_c) v_c
+ * with K(i) the union of the key blocks kept for r's query block i (list row h*nq+i).
+ *   q, k, v, o : bf16 [H, N, D]; D in {64, 128}; list->block in {64, 128};
+ *                list->nq == list->nk == ceil(N/B).
+ *   lse_opt    : NULL or fp32 [H, N], natural-log LSE over the kept keys.
+ *   scale      : > 0 (typically 1/sqrt(D)).
+ *   flags      : 0, or CALIB_ATTN_OUT_F32 to write o as fp32 (no output rounding).
+ * Arithmetic: S = QK^T and O += PV on the tensor cores with fp32 accumulation; P is
+ * rounded to bf16 for the PV product and O is divided by the sum of those rounded
+ * weights.
+ * A row with no kept block writes O = 0 and LSE = -inf.  With an all-kept list this is
+ * dense attention. */
+calib_status sparse_attn_fwd(const void* q, const void* k, const void* v, void* o,
+                             float* lse_opt, int H, int N, int D, float scale,
+                             const calib_block_list* list, uint32_t flags, void* stream);
+
+/* Block-sparse attention with spatial repetition ([zh] §2.2B, [fr] §2.C): heads flagged
+ * in head_repeat (HOST uint8 [H]) compute only their anchor tokens (calib_anchor_rows
+ * order) and write each anchor's output (and LSE) to every token it stands for -- token
+ * (f, y, x) takes anchor (f, floor(y/stride)*stride, x); text tokens are their own
+ * anchors.  For a flagged head, list rows i < ceil(N_a/B) are in anchor block space and
+ * rows beyond are ignored; unflagged heads behave as in sparse_attn_fwd.
+ * N = F*Hl*Wl + n_text; q, k, v, o, lse_opt, D, scale and flags as in sparse_attn_fwd.
+ * H <= 1024, stride >= 1 (stride 1 makes every token its own anchor). */
+calib_status sparse_attn_fwd_repeat(const void* q, const void* k, const void* v, void* o,
+                                    float* lse_opt, int H, int D, int F, int Hl, int Wl,
+                                    int n_text, int stride, const uint8_t* head_repeat,
+                                    float scale, const calib_block_list* list,
+                                    uint32_t flags, void* stream);
+
+/* Failure-detection self-test: launches one kernel that waits, with the library's bounded
+ * wait, on an mbarrier that nothing ever completes, giving up after timeout_us
+ * microseconds.  Returns what calib_device_check then reports: CALIB_ERR_TIMEOUT when
+ * the bound works (the GPU context stays usable).  Synchronises `stream`. */
+calib_status calib_selftest_wait_timeout(uint32_t timeout_us, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CALIBATT_H */

@@ -1,0 +1,401 @@
+"""GPU parity: every CUDA entry point against the float64 oracle on the same seeded inputs.
+
+Bars (from the method's tolerance statement): masks, CSR lists, schedules and anchor
+lists bit-exact (selection run from identical fp32 energies); block energies within
+1e-4 relative (below a floor of 1e-12 * |I_i|, within 1e-16 * |I_i| absolute, since fp32
+exp underflows far above fp64's range); attention outputs from bf16 inputs with fp32
+accumulation within 2e-2 max-abs and 2e-3 mean-relative (mean |dO| / mean |O_ref|) of the
+fp64 result.  That bar applies as stated to the fp32-output mode.  A bf16 output adds its
+own rounding, up to half a bf16 ulp of the value (0.031 at |O| in [8, 16)), so bf16
+outputs are held to 2e-2 + ulp_bf16(|O_ref|)/2 elementwise and the same 2e-3 mean-relative.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from calibrated_block_sparse_calib_b200 import ops, synth
+from conftest import to64
+
+pytestmark = pytest.mark.gpu
+
+ATTN_MAXABS = 2e-2
+ATTN_MEANREL = 2e-3
+E_REL = 1e-4
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _need_cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    ops.lib()
+
+
+def _shape(H, D, F, Hl, Wl, B, n_text=0, rank=8):
+    return synth.Workload("adhoc", synth.VideoShape(H=H, D=D, F=F, Hl=Hl, Wl=Wl, n_text=n_text, block=B),
+                          rank=rank)
+
+
+def _inputs(wl, seed, device="cuda"):
+    q, k, v = synth.make_qkv(wl, seed=seed)
+    return q.to(device), k.to(device), v.to(device)
+
+
+def half_ulp_bf16(x):
+    """Half a bf16 ulp at |x| (8 significant bits): 2^(floor(log2 |x|) - 8)."""
+    ax = np.maximum(np.abs(x), 2.0 ** -126)
+    return np.ldexp(1.0, np.floor(np.log2(ax)).astype(np.int64) - 8)
+
+
+def check_attn(o_gpu, o_ref, rows=None):
+    og = to64(o_gpu)
+    if rows is not None:
+        og, o_ref = og[:, rows], o_ref[:, rows]
+    d = np.abs(og - o_ref)
+    allow = ATTN_MAXABS + (half_ulp_bf16(o_ref) if o_gpu.dtype == torch.bfloat16 else 0.0)
+    excess = float((d - allow).max())
+    maxabs = float(d.max())
+    meanrel = float(d.mean() / np.abs(o_ref).mean())
+    assert excess <= 0 and meanrel <= ATTN_MEANREL, (maxabs, excess, meanrel)
+    return maxabs, meanrel
+
+
+def check_energy(e_gpu, e_ref, Nq, B):
+    eg = to64(e_gpu)
+    nq = e_ref.shape[1]
+    rows = np.array([min((i + 1) * B, Nq) - i * B for i in range(nq)], float)[None, :, None]
+    floor = 1e-12 * rows
+    big = e_ref >= floor
+    err = np.abs(eg - e_ref)
+    assert np.all(err[big] <= E_REL * e_ref[big]), float((err[big] / e_ref[big]).max())
+    assert np.all(err[~big] <= 1e-16 * np.broadcast_to(rows, e_ref.shape)[~big])
+    return float((err[big] / e_ref[big]).max())
+
+
+def _blist(mask_np, B, schedule=True):
+    return ops.BlockList.from_mask(torch.from_numpy(mask_np).cuda(), B, schedule=schedule)
+
+
+def _rand_mask(rng, H, nq, nk, p=0.4, diag=True):
+    m = (rng.random((H, nq, nk)) < p).astype(np.uint8)
+    if diag:
+        for i in range(nq):
+            m[:, i, min(i, nk - 1)] = 1
+    return m
+
+
+# ------------------------------------------------------------------------------------
+# integer kernels: bit-exact
+# ------------------------------------------------------------------------------------
+
+def _energy_rows(rng, H, nq, nk):
+    e = np.empty((H, nq, nk), np.float64)
+    for h in range(H):
+        for i in range(nq):
+            kind = (h * nq + i) % 6
+            if kind == 0:
+                x = rng.random(nk)
+            elif kind == 1:
+                x = rng.exponential(size=nk) ** 4
+            elif kind == 2:
+                x = np.round(rng.random(nk) * 4) / 4
+            elif kind == 3:
+                x = np.exp(-40 * rng.random(nk))
+            elif kind == 4:
+                x = rng.random(nk) * 1e-39            # fp32 subnormal range
+            else:
+                x = np.zeros(nk)
+                x[rng.integers(0, nk)] = 1.0
+            e[h, i] = x
+    return e.astype(np.float32)
+
+
+@pytest.mark.parametrize("nk", [1, 7, 64, 256, 591, 1024])
+@pytest.mark.parametrize("tau", [1e-7, 0.9, 0.95, 0.99, 1.0])
+def test_select_bit_exact(nk, tau):
+    rng = np.random.default_rng(nk * 31 + int(tau * 1000))
+    H, nq = 2, 6
+    e = _energy_rows(rng, H, nq, nk)
+    e[1, 5] = 0.0                                                  # an all-zero row
+    ref = oracle.select_mask(e, tau)
+    got = ops.select_mask(torch.from_numpy(e).cuda(), tau).cpu().numpy()
+    np.testing.assert_array_equal(got, ref)
+
+
+def test_select_forced_and_count_accumulation():
+    rng = np.random.default_rng(5)
+    H, nq, nk = 3, 5, 100
+    counts = torch.zeros(H, nq, nk, dtype=torch.int32, device="cuda")
+    acc = np.zeros((H, nq, nk), np.int64)
+    for d in range(3):
+        e = _energy_rows(rng, H, nq, nk)
+        force = (rng.random((H, nq, nk)) < 0.05).astype(np.uint8)
+        ref = oracle.select_mask(e, 0.9, force_keep=force)
+        got = ops.select_mask(torch.from_numpy(e).cuda(), 0.9, force_keep=torch.from_numpy(force).cuda(),
+                              count_accum=counts).cpu().numpy()
+        np.testing.assert_array_equal(got, ref)
+        acc += ref
+    np.testing.assert_array_equal(counts.cpu().numpy(), acc)
+
+
+@pytest.mark.parametrize("n_inputs,rho", [(1, (1, 2)), (3, (1, 2)), (4, (1, 2)), (5, (1, 3)), (4, (0, 1))])
+def test_aggregate_bit_exact(n_inputs, rho):
+    rng = np.random.default_rng(n_inputs * 7 + rho[0])
+    c = rng.integers(0, n_inputs + 1, size=(3, 9, 70)).astype(np.int32)
+    c[1, 3] = 0
+    c[1, 3, 5] = 1                                                   # a row the vote may empty
+    ref = oracle.aggregate_masks(c, n_inputs, *rho)
+    got = ops.aggregate_masks(torch.from_numpy(c).cuda(), n_inputs, rho).cpu().numpy()
+    np.testing.assert_array_equal(got, ref)
+
+
+@pytest.mark.parametrize("H,nq,nk", [(1, 1, 1), (2, 8, 8), (3, 37, 53), (40, 158, 591)])
+def test_csr_and_schedule_bit_exact(H, nq, nk):
+    rng = np.random.default_rng(H * nq + nk)
+    m = _rand_mask(rng, H, nq, nk, p=0.3, diag=False)
+    if H * nq > 2:
+        m[0, nq - 1] = 0                                              # an empty row
+    rp_ref, ci_ref = oracle.mask_to_csr(m)
+    rp, ci = ops.mask_to_csr(torch.from_numpy(m).cuda())
+    rp = rp.cpu().numpy()
+    np.testing.assert_array_equal(rp, rp_ref)
+    np.testing.assert_array_equal(ci.cpu().numpy()[: rp[-1]], ci_ref)
+    w = ops.build_schedule(torch.from_numpy(rp).cuda(), H, nq).cpu().numpy()
+    np.testing.assert_array_equal(w, oracle.build_schedule(rp_ref, H, nq))
+
+
+@pytest.mark.parametrize("geom", [(4, 8, 16, 0, 2), (21, 45, 80, 0, 4), (28, 30, 53, 256, 4), (3, 7, 5, 9, 3),
+                                  (2, 5, 3, 0, 1)])
+def test_anchor_rows_exact(geom):
+    got = ops.anchor_rows(*geom).cpu().numpy()
+    np.testing.assert_array_equal(got, oracle.anchor_rows(*geom))
+
+
+# ------------------------------------------------------------------------------------
+# block energies
+# ------------------------------------------------------------------------------------
+
+def test_energy_tiny_all_inputs(tiny_inputs):
+    wl, qkv = tiny_inputs
+    B, D = wl.shape.block, wl.shape.D
+    scale = 1.0 / math.sqrt(D)
+    for q, k, _ in qkv:
+        ref = oracle.block_energy(to64(q), to64(k), scale, B)
+        got = ops.block_energy(q.cuda(), k.cuda(), B)
+        check_energy(got, ref, wl.shape.N, B)
+
+
+@pytest.mark.parametrize("D,B,geom", [(128, 128, (5, 10, 20)), (128, 64, (3, 9, 11)), (64, 128, (2, 13, 17))])
+def test_energy_ragged(D, B, geom):
+    wl = _shape(2, D, *geom, B)
+    q, k, _ = _inputs(wl, seed=100 + D + B)
+    scale = 1.0 / math.sqrt(D)
+    ref = oracle.block_energy(to64(q), to64(k), scale, B)
+    got = ops.block_energy(q, k, B)
+    check_energy(got, ref, wl.shape.N, B)
+
+
+def test_energy_cached_lse_and_accumulate(tiny_inputs):
+    wl, qkv = tiny_inputs
+    B, D = wl.shape.block, wl.shape.D
+    scale = 1.0 / math.sqrt(D)
+    q, k, _ = qkv[1]
+    lse = oracle.row_lse(to64(q), to64(k), scale)
+    ref = oracle.block_energy(to64(q), to64(k), scale, B, lse=lse)
+    lse_t = torch.from_numpy(lse.astype(np.float32)).cuda()
+    got = ops.block_energy(q.cuda(), k.cuda(), B, lse=lse_t)
+    check_energy(got, ref, wl.shape.N, B)
+    acc = ops.block_energy(q.cuda(), k.cuda(), B, accumulate=True)
+    acc = ops.block_energy(q.cuda(), k.cuda(), B, out=acc, accumulate=True)
+    check_energy(acc, 2 * ref, wl.shape.N, B)
+
+
+def test_energy_anchor_rows(tiny_inputs):
+    wl, qkv = tiny_inputs
+    s = wl.shape
+    B = s.block
+    q, k, _ = qkv[0]
+    rows = oracle.anchor_rows(s.F, s.Hl, s.Wl, 0, 2)
+    ref = oracle.block_energy(to64(q), to64(k), 1.0 / math.sqrt(s.D), B, q_rows=rows)
+    q_rows = ops.anchor_rows(s.F, s.Hl, s.Wl, 0, 2)
+    got = ops.block_energy(q.cuda(), k.cuda(), B, q_rows=q_rows)
+    check_energy(got, ref, len(rows), B)
+
+
+# ------------------------------------------------------------------------------------
+# attention
+# ------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
+def test_attention_tiny_random_and_dense(tiny_inputs, out_dtype):
+    wl, qkv = tiny_inputs
+    B, D, N = wl.shape.block, wl.shape.D, wl.shape.N
+    scale = 1.0 / math.sqrt(D)
+    q, k, v = qkv[0]
+    rng = np.random.default_rng(1)
+    nb = wl.shape.nblk
+    for m in (_rand_mask(rng, 2, nb, nb, 0.4), np.ones((2, nb, nb), np.uint8)):
+        O_ref, L_ref = oracle.sparse_attention(to64(q), to64(k), to64(v), scale, B, m)
+        O, L = ops.sparse_attn_fwd(q.cuda(), k.cuda(), v.cuda(), _blist(m, B), return_lse=True,
+                                   out_dtype=out_dtype)
+        assert O.dtype == out_dtype
+        check_attn(O, O_ref)
+        np.testing.assert_allclose(to64(L), L_ref, rtol=0, atol=2e-4)
+
+
+@pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("D,B,geom,p", [(128, 128, (5, 10, 20), 0.35), (128, 64, (3, 9, 11), 0.5),
+                                        (64, 128, (2, 13, 17), 0.6), (128, 128, (1, 1, 70), 1.0),
+                                        (128, 128, (3, 17, 40), 0.2)])
+def test_attention_ragged(D, B, geom, p, out_dtype):
+    wl = _shape(3, D, *geom, B)
+    q, k, v = _inputs(wl, seed=200 + D + B + geom[2])
+    nb = wl.shape.nblk
+    m = _rand_mask(np.random.default_rng(geom[2]), 3, nb, nb, p)
+    O_ref, L_ref = oracle.sparse_attention(to64(q), to64(k), to64(v), 1.0 / math.sqrt(D), B, m)
+    O, L = ops.sparse_attn_fwd(q, k, v, _blist(m, B), return_lse=True, out_dtype=out_dtype)
+    check_attn(O, O_ref)
+    np.testing.assert_allclose(to64(L), L_ref, rtol=0, atol=2e-4)
+
+
+def test_attention_empty_rows_write_zero():
+    wl = _shape(2, 128, 2, 8, 30, 128)
+    q, k, v = _inputs(wl, seed=300)
+    nb = wl.shape.nblk
+    m = _rand_mask(np.random.default_rng(3), 2, nb, nb, 0.5)
+    m[0, 1] = 0
+    m[1, nb - 1] = 0
+    O_ref, _ = oracle.sparse_attention(to64(q), to64(k), to64(v), 1 / math.sqrt(128), 128, m)
+    O, L = ops.sparse_attn_fwd(q, k, v, _blist(m, 128), return_lse=True)
+    O = O.cpu()
+    assert torch.all(O[0, 128:256] == 0) and torch.all(torch.isneginf(L[0, 128:256].cpu()))
+    check_attn(O, O_ref)
+
+
+def test_masked_blocks_do_not_matter_bitwise():
+    wl = _shape(2, 128, 4, 8, 24, 128)
+    q, k, v = _inputs(wl, seed=400)
+    nb = wl.shape.nblk
+    m = _rand_mask(np.random.default_rng(4), 2, nb, nb, 0.3)
+    m[:, :, 2] = 0
+    bl = _blist(m, 128)
+    O1 = ops.sparse_attn_fwd(q, k, v, bl)
+    k2, v2 = k.clone(), v.clone()
+    k2[:, 256:384] = torch.randn_like(k2[:, 256:384].float()).to(torch.bfloat16) * 5
+    v2[:, 256:384] = torch.randn_like(v2[:, 256:384].float()).to(torch.bfloat16) * 5
+    O2 = ops.sparse_attn_fwd(q, k2, v2, bl)
+    assert torch.equal(O1, O2)
+    # processing order does not change any output bit
+    O3 = ops.sparse_attn_fwd(q, k, v, _blist(m, 128, schedule=False))
+    assert torch.equal(O1, O3)
+
+
+def test_repeat_tiny(tiny_inputs):
+    wl, qkv = tiny_inputs
+    s = wl.shape
+    B = s.block
+    q, k, v = qkv[2]
+    nb = s.nblk
+    rng = np.random.default_rng(6)
+    m = _rand_mask(rng, 2, nb, nb, 0.5)
+    nqa = synth.anchor_block_count(s, 2)
+    m[1, nqa:] = 0
+    rep = [False, True]
+    O_ref, L_ref = oracle.sparse_attention_repeat(to64(q), to64(k), to64(v), 1 / math.sqrt(s.D), B, m, rep,
+                                                  s.F, s.Hl, s.Wl, 0, 2)
+    O, L = ops.sparse_attn_fwd_repeat(q.cuda(), k.cuda(), v.cuda(), _blist(m, B), rep, s.F, s.Hl, s.Wl, 0, 2,
+                                      return_lse=True)
+    check_attn(O, O_ref)
+    np.testing.assert_allclose(to64(L), L_ref, rtol=0, atol=2e-4)
+    Oc = O.cpu()
+    for t in range(s.N):                       # each row of the repeat head equals its anchor's
+        a = oracle.anchor_rows(s.F, s.Hl, s.Wl, 0, 2)[oracle.anchor_index_of_token(t, s.F, s.Hl, s.Wl, 0, 2)]
+        assert torch.equal(Oc[1, t], Oc[1, int(a)])
+
+
+@pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("stride", [1, 3, 4])
+def test_repeat_with_text_and_ragged_groups(stride, out_dtype):
+    wl = _shape(3, 128, 3, 7, 20, 128, n_text=40)
+    s = wl.shape
+    q, k, v = _inputs(wl, seed=500 + stride)
+    nb = s.nblk
+    m = _rand_mask(np.random.default_rng(stride), 3, nb, nb, 0.5)
+    nqa = synth.anchor_block_count(s, stride)
+    rep = [True, False, True]
+    for h in (0, 2):
+        m[h, nqa:] = 0
+    O_ref, L_ref = oracle.sparse_attention_repeat(to64(q), to64(k), to64(v), 1 / math.sqrt(128), 128, m, rep,
+                                                  s.F, s.Hl, s.Wl, s.n_text, stride)
+    O, L = ops.sparse_attn_fwd_repeat(q, k, v, _blist(m, 128), rep, s.F, s.Hl, s.Wl, s.n_text, stride,
+                                      return_lse=True, out_dtype=out_dtype)
+    check_attn(O, O_ref)
+    np.testing.assert_allclose(to64(L), L_ref, rtol=0, atol=2e-4)
+
+
+# ------------------------------------------------------------------------------------
+# the whole calibration + inference pipeline at the tiny workload
+# ------------------------------------------------------------------------------------
+
+def test_calibration_pipeline_tiny(tiny_inputs):
+    wl, qkv = tiny_inputs
+    s = wl.shape
+    B = s.block
+    tau = wl.extra["tau"]
+    rho = wl.extra["rho"]
+    scale = 1.0 / math.sqrt(s.D)
+    nb = s.nblk
+    counts = torch.zeros(s.H, nb, nb, dtype=torch.int32, device="cuda")
+    cnt_ref = np.zeros((s.H, nb, nb), np.int64)
+    energies_gpu = []
+    for q, k, _ in qkv:
+        e_gpu = ops.block_energy(q.cuda(), k.cuda(), B)
+        e_ref = oracle.block_energy(to64(q), to64(k), scale, B)
+        check_energy(e_gpu, e_ref, s.N, B)
+        energies_gpu.append(e_gpu.cpu().numpy())
+        # selection from identical (GPU) energies: bit-exact
+        m_gpu = ops.select_mask(e_gpu, tau, count_accum=counts).cpu().numpy()
+        np.testing.assert_array_equal(m_gpu, oracle.select_mask(e_gpu.cpu().numpy(), tau))
+        cnt_ref += m_gpu
+    np.testing.assert_array_equal(counts.cpu().numpy(), cnt_ref)
+    agg = ops.aggregate_masks(counts, len(qkv), rho).cpu().numpy()
+    np.testing.assert_array_equal(agg, oracle.aggregate_masks(cnt_ref, len(qkv), *rho))
+    # energy-mean mode: the sum of fp32 energies is what selection sees
+    bl = _blist(agg, B)
+    q, k, v = qkv[0]
+    O_ref, _ = oracle.sparse_attention(to64(q), to64(k), to64(v), scale, B, agg)
+    check_attn(ops.sparse_attn_fwd(q.cuda(), k.cuda(), v.cuda(), bl), O_ref)
+
+
+# ------------------------------------------------------------------------------------
+# full-size Wan-1.3B-shaped call, sampled query blocks (the bench's launch configuration)
+# ------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
+def test_wan13b_sampled_blocks(out_dtype):
+    wl = synth.WORKLOADS["wan13b"]
+    s = wl.shape
+    q, k, v = synth.make_qkv(wl, device="cuda")
+    mask = synth.make_head_masks(wl)
+    bl = _blist(mask, s.block)
+    O = ops.sparse_attn_fwd(q, k, v, bl, out_dtype=out_dtype)
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(11)
+    blocks = sorted(set(rng.choice(s.nblk - 1, size=7, replace=False).tolist()) | {s.nblk - 1})
+    rows = np.concatenate([np.arange(i * s.block, min((i + 1) * s.block, s.N)) for i in blocks])
+    heads = [0, 5, 11]
+    qh, kh, vh = (to64(t[heads]) for t in (q, k, v))
+    O_ref, _ = oracle.sparse_attention(qh, kh, vh, 1 / math.sqrt(s.D), s.block, mask[heads], q_blocks=blocks)
+    check_attn(O[heads], O_ref, rows=rows)
+
+
+def test_wait_timeout_selftest_keeps_context_usable(tiny_inputs):
+    assert ops.selftest_wait_timeout(2000) == ops.CALIB_ERR_TIMEOUT
+    ops.device_check()                                   # the status word was cleared
+    wl, qkv = tiny_inputs
+    q, k, _ = qkv[0]
+    e = ops.block_energy(q.cuda(), k.cuda(), wl.shape.block)
+    ops.device_check()
+    assert torch.isfinite(e).all()
