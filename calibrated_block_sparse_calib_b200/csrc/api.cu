@@ -95,15 +95,22 @@ calib_status launch_status() {
 }
 
 // ---- attention ---------------------------------------------------------------------
-template <int D, int BLK>
+template <int D, int BLK, bool WITH_LSE>
 calib_status launch_attn(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                          const calib::AttnParams& p, int grid, cudaStream_t st) {
     constexpr int KST = 2, VST = 2;
     using L = calib::AttnSmem<D, BLK, KST, VST>;
-    auto* fn = calib::attn_fwd_kernel<D, BLK, KST, VST>;
+    auto* fn = calib::attn_fwd_kernel<D, BLK, KST, VST, WITH_LSE>;
     if (calib_status s = ensure_smem(reinterpret_cast<const void*>(fn), L::BYTES)) return s;
     fn<<<grid, calib::kAttnThreads, L::BYTES, st>>>(tq, tk, tv, p);
     return launch_status();
+}
+
+template <int D, int BLK>
+calib_status launch_attn_lse(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                             const calib::AttnParams& p, int grid, cudaStream_t st) {
+    return p.lse ? launch_attn<D, BLK, true>(tq, tk, tv, p, grid, st)
+                 : launch_attn<D, BLK, false>(tq, tk, tv, p, grid, st);
 }
 
 calib_status attn_common(const void* q, const void* k, const void* v, void* o, float* lse, int H, int N,
@@ -147,9 +154,10 @@ calib_status attn_common(const void* q, const void* k, const void* v, void* o, f
         !make_tmap(&tv, v, D, N, H, B))
         return CALIB_ERR_CUDA;
     cudaStream_t st = as_stream(stream);
-    if (D == 128) return B == 128 ? launch_attn<128, 128>(tq, tk, tv, p, grid, st)
-                                  : launch_attn<128, 64>(tq, tk, tv, p, grid, st);
-    return B == 128 ? launch_attn<64, 128>(tq, tk, tv, p, grid, st) : launch_attn<64, 64>(tq, tk, tv, p, grid, st);
+    if (D == 128) return B == 128 ? launch_attn_lse<128, 128>(tq, tk, tv, p, grid, st)
+                                  : launch_attn_lse<128, 64>(tq, tk, tv, p, grid, st);
+    return B == 128 ? launch_attn_lse<64, 128>(tq, tk, tv, p, grid, st)
+                    : launch_attn_lse<64, 64>(tq, tk, tv, p, grid, st);
 }
 
 // ---- energy ------------------------------------------------------------------------
@@ -269,7 +277,7 @@ calib_status calib_build_schedule(const int32_t* row_ptr, int H, int nq, int32_t
     if (calib_status s = check_device()) return s;
     const int bytes = calib::kSchedBins * 4;
     if (calib_status s = ensure_smem(reinterpret_cast<const void*>(calib::schedule_kernel), bytes)) return s;
-    calib::schedule_kernel<<<1, 1024, bytes, as_stream(stream)>>>(row_ptr, H * nq, nq, work_out);
+    calib::schedule_kernel<<<H, 1024, bytes, as_stream(stream)>>>(row_ptr, nq, work_out);
     return launch_status();
 }
 

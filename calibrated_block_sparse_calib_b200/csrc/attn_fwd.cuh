@@ -8,16 +8,23 @@
 // broadcast to the other rows of their frame ([zh] §2.2B, [fr] §2.C).
 //
 // One CTA per work item (head h, query block i).  192 threads:
-//   warp 0      TMA producer: Q tile once (or nothing for repeat heads, whose anchor
-//               rows are gathered by the softmax warps), then K_j / V_j for each kept j
-//               through KST / VST-deep rings.
+//   warp 0      TMA producer: Q tile once (repeat heads: nothing, their anchor rows are
+//               gathered by the softmax warps), then K_j / V_j for each kept j through
+//               KST / VST-deep rings (K runs one tile ahead of V).
 //   warp 1      TMEM owner (512 columns) and single-thread MMA issuer:
-//               S_t = Q K_j^T  (SS MMA, M=128, N=B, K=D) into S buffer t%2,
-//               O  += P_t V_j  (TS MMA: P from TMEM, V from SMEM, M=128, N=D, K=B).
-//   warps 2..5  softmax + epilogue, one query row per thread (TMEM lane = row):
-//               online max/sum in the log2 domain with lazy rescaling of O, P written
-//               back to TMEM as bf16 over S's columns, final 1/l, bf16 stores.
-// Tensor memory: S0 = cols [0,128), S1 = [128,256), O = [256, 256+D).
+//               S_t = Q K_j^T        SS MMA, M=128, N=B, K=D, into S buffer t%2;
+//               [O|l] += P_t [V_j|1] TS MMA, M=128, N=D+16, K=B: P from TMEM, V from SMEM.
+//               The 16 extra B columns are a constant all-ones chunk placed after each V
+//               stage, so column D of the accumulator is the row sum of the bf16 P that
+//               entered the product (the softmax normaliser, exactly consistent with O).
+//   warps 2..5  softmax + epilogue, one query row per thread (TMEM lane = row): online
+//               row max in the log2 domain with lazy rescaling (O is rescaled only when the
+//               max grows by more than 2^8), P = 2^(x - m) written back over S as bf16,
+//               final division by the accumulated row sum, bf16 (or fp32) stores.
+// Each row's key list is walked starting at its diagonal block (the first kept key block
+// at or after the query block), where local attention peaks, so the running max is
+// usually final after the first tile and O is rarely rescaled.
+// Tensor memory: S0 = cols [0,128), S1 = [128,256), [O|l] = [256, 256+D+16).
 #pragma once
 #include <cuda_bf16.h>
 #include "ptx.cuh"
@@ -28,6 +35,7 @@ constexpr int kAttnThreads = 192;
 constexpr int kTileM = 128;               // query rows per tile (MMA M)
 constexpr float kRescaleLog2 = 8.0f;      // rescale O only when the row max grows by > 2^8
 constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kTmemO = 256;          // first column of the [O | rowsum] accumulator
 
 struct AttnParams {
     const __nv_bfloat16* q;   // [H, N, D] (read directly only for repeat-head gathers)
@@ -73,39 +81,47 @@ __device__ __forceinline__ void gather_q_row(uint8_t* sQ, int r, const __nv_bflo
     }
 }
 
-// Write one output row (D values already scaled, fp32 in registers, 32 per chunk).
-__device__ __forceinline__ void store_row_chunk(__nv_bfloat16* dst, const uint32_t (&packed)[16]) {
+// Write 32 output values of one row (already normalised).
+__device__ __forceinline__ void store_row32_bf16(__nv_bfloat16* dst, const uint32_t (&packed)[16]) {
     uint4* d = reinterpret_cast<uint4*>(dst);
 #pragma unroll
     for (int v = 0; v < 4; ++v)
         d[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
 }
+__device__ __forceinline__ void store_row32_f32(float* dst, const uint32_t* raw) {
+    uint4* d = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+    for (int v = 0; v < 8; ++v) d[v] = make_uint4(raw[4 * v], raw[4 * v + 1], raw[4 * v + 2], raw[4 * v + 3]);
+}
 
 template <int D, int BLK, int KST, int VST>
 struct AttnSmem {
     static constexpr int CH = D / 64;                     // 128-byte chunks per row
+    static constexpr uint32_t CHUNK = BLK * 128;          // one 64-column chunk of a K/V tile
     static constexpr uint32_t Q_BYTES = CH * kTileM * 128;
-    static constexpr uint32_t KV_BYTES = CH * BLK * 128;
+    static constexpr uint32_t K_BYTES = CH * CHUNK;
+    static constexpr uint32_t V_STAGE = (CH + 1) * CHUNK; // V chunks + the all-ones chunk
     static constexpr uint32_t OFF_K = Q_BYTES;
-    static constexpr uint32_t OFF_V = OFF_K + KST * KV_BYTES;
-    static constexpr uint32_t OFF_BAR = OFF_V + VST * KV_BYTES;
+    static constexpr uint32_t OFF_V = OFF_K + KST * K_BYTES;
+    static constexpr uint32_t OFF_BAR = OFF_V + VST * V_STAGE;
     // barrier indices
     static constexpr int B_Q = 0, B_KF = 1, B_KE = B_KF + KST, B_VF = B_KE + KST,
                          B_VE = B_VF + VST, B_SF = B_VE + VST, B_PF = B_SF + 2, B_O = B_PF + 2,
                          B_DRAIN = B_O + 1, NBARS = B_DRAIN + 1;
-    static constexpr uint32_t OFF_MISC = OFF_BAR + NBARS * 8;
+    static constexpr uint32_t OFF_MISC = OFF_BAR + NBARS * 8;   // tmem base, abort flag, t0
     // + alignment slack; at least 120 KB so that one CTA (holding all 512 TMEM columns)
     // is resident per SM and no CTA waits in tcgen05.alloc.
     static constexpr uint32_t RAW = OFF_MISC + 16 + 1024;
     static constexpr uint32_t BYTES = RAW > 120u * 1024 ? RAW : 120u * 1024;
 };
 
-template <int D, int BLK, int KST, int VST>
+template <int D, int BLK, int KST, int VST, bool WITH_LSE>
 __global__ void __launch_bounds__(kAttnThreads, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
     using L = AttnSmem<D, BLK, KST, VST>;
     constexpr int CH = L::CH;
+    constexpr int NPV = D + 16;                            // PV MMA N: O columns + row sum
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
@@ -116,6 +132,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     auto bar = [&](int idx) -> uint32_t { return bar0 + 8u * idx; };
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
+    int* t0_slot = reinterpret_cast<int*>(smem + L::OFF_MISC + 8);
 
     const uint32_t warp = warp_id(), lane = lane_id();
 
@@ -145,6 +162,13 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         mbar_init(bar(L::B_O), 1);
         mbar_init(bar(L::B_DRAIN), 1);
         *abort_flag = 0;
+        // walk the list from the diagonal block: first kept key block at or after the
+        // key block holding the query block's first token
+        const int tok = rep ? anchor_token(p, min(i * BLK, Nq - 1)) : i * BLK;
+        const int jd = tok / BLK;
+        int t0 = 0;
+        while (t0 < nkept && p.col_idx[kbeg + t0] < jd) ++t0;
+        *t0_slot = t0 < nkept ? t0 : 0;
         fence_barrier_init();
     }
     if (warp == 0 && lane == 0) {
@@ -156,11 +180,28 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         tmem_alloc(smem_u32(tmem_slot), kTmemCols);
         tmem_relinquish();
     }
+    if (warp >= 2) {
+        // all-ones chunk after every V stage: bf16 1.0 = 0x3F80 (the swizzle is
+        // irrelevant for a constant tile)
+        const uint4 ones = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
+        for (int s = 0; s < VST; ++s) {
+            uint4* dst = reinterpret_cast<uint4*>(sV + s * L::V_STAGE + CH * L::CHUNK);
+            for (int x = static_cast<int>(threadIdx.x) - 64; x < static_cast<int>(L::CHUNK / 16); x += 128)
+                dst[x] = ones;
+        }
+        fence_proxy_async_smem();
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    const int t0 = *t0_slot;
     const WaitCtl ctl{abort_flag, p.timeout_ns};
+    // list position of step t (rotated to start at the diagonal block)
+    auto kidx = [&](int t) -> int {
+        const int u = t + t0;
+        return kbeg + (u >= nkept ? u - nkept : u);
+    };
 
     // bookkeeping for the abort drain (producer only)
     int armed_q = 0, armed_k[KST], armed_v[VST];
@@ -181,26 +222,25 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             auto issue_k = [&](int t) -> bool {
                 const int s = t % KST;
                 if (!mbar_wait(bar(L::B_KE + s), ((t / KST) & 1) ^ 1, ctl)) return false;
-                const int j = p.col_idx[kbeg + t];
-                mbar_arrive_expect_tx(bar(L::B_KF + s), L::KV_BYTES);
+                const int j = p.col_idx[kidx(t)];
+                mbar_arrive_expect_tx(bar(L::B_KF + s), L::K_BYTES);
                 for (int c = 0; c < CH; ++c)
-                    tma_load_3d(smem_u32(sK + s * L::KV_BYTES + c * BLK * 128), &tm_k, bar(L::B_KF + s),
-                                c * 64, j * BLK, h);
+                    tma_load_3d(smem_u32(sK + s * L::K_BYTES + c * L::CHUNK), &tm_k, bar(L::B_KF + s), c * 64,
+                                j * BLK, h);
                 ++armed_k[s];
                 return true;
             };
             auto issue_v = [&](int t) -> bool {
                 const int s = t % VST;
                 if (!mbar_wait(bar(L::B_VE + s), ((t / VST) & 1) ^ 1, ctl)) return false;
-                const int j = p.col_idx[kbeg + t];
-                mbar_arrive_expect_tx(bar(L::B_VF + s), L::KV_BYTES);
+                const int j = p.col_idx[kidx(t)];
+                mbar_arrive_expect_tx(bar(L::B_VF + s), L::K_BYTES);
                 for (int c = 0; c < CH; ++c)
-                    tma_load_3d(smem_u32(sV + s * L::KV_BYTES + c * BLK * 128), &tm_v, bar(L::B_VF + s),
-                                c * 64, j * BLK, h);
+                    tma_load_3d(smem_u32(sV + s * L::V_STAGE + c * L::CHUNK), &tm_v, bar(L::B_VF + s), c * 64,
+                                j * BLK, h);
                 ++armed_v[s];
                 return true;
             };
-            // K runs ahead of V: the MMA order is QK_0, QK_1, PV_0, QK_2, PV_1, ...
             bool ok = issue_k(0);
             for (int t = 0; ok && t < nkept; ++t) {
                 if (t + 1 < nkept) ok = issue_k(t + 1);
@@ -211,7 +251,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         // ===================== MMA issuer =====================
         if (lane == 0 && nkept > 0) {
             constexpr uint32_t idesc_qk = idesc_bf16_f32(kTileM, BLK, false, false);
-            constexpr uint32_t idesc_pv = idesc_bf16_f32(kTileM, D, false, true);
+            constexpr uint32_t idesc_pv = idesc_bf16_f32(kTileM, NPV, false, true);
             const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV);
             bool ok = mbar_wait(bar(L::B_Q), 0, ctl);
             tc_fence_after();
@@ -225,7 +265,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     const uint32_t inner = (kk & 3) * 32;   // K step of 16 bf16 inside a 128-B atom
                     const uint64_t ad = smem_desc_sw128(sQa + (kk >> 2) * kTileM * 128 + inner, 16, 1024);
                     const uint64_t bd =
-                        smem_desc_sw128(sKa + s * L::KV_BYTES + (kk >> 2) * BLK * 128 + inner, 16, 1024);
+                        smem_desc_sw128(sKa + s * L::K_BYTES + (kk >> 2) * L::CHUNK + inner, 16, 1024);
                     umma_ss(d_tmem, ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
                 }
                 umma_commit(bar(L::B_SF + (t & 1)));
@@ -248,9 +288,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 const uint32_t a_tmem = tmem + (t & 1) * 128;
 #pragma unroll
                 for (int kk = 0; kk < BLK / 16; ++kk) {
-                    const uint64_t bd =
-                        smem_desc_sw128(sVa + sv * L::KV_BYTES + kk * 16 * 128, BLK * 128, 1024);
-                    umma_ts(tmem + 256, a_tmem + kk * 8, bd, idesc_pv, (t > 0 || kk > 0) ? 1u : 0u);
+                    const uint64_t bd = smem_desc_sw128(sVa + sv * L::V_STAGE + kk * 16 * 128, L::CHUNK, 1024);
+                    umma_ts(tmem + kTmemO, a_tmem + kk * 8, bd, idesc_pv, (t > 0 || kk > 0) ? 1u : 0u);
                 }
                 umma_commit(bar(L::B_O));
                 umma_commit(bar(L::B_VE + sv));
@@ -269,67 +308,82 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             fence_proxy_async_smem();
             mbar_arrive(bar(L::B_Q));
         }
-        float m_run = -INFINITY, l_run = 0.f, lq_run = 0.f;
+        const float sc = p.scale_log2;
+        float m_run = -INFINITY, l_run = 0.f;
         bool ok = true;
         for (int t = 0; t < nkept; ++t) {
-            const int j = p.col_idx[kbeg + t];
+            const int j = p.col_idx[kidx(t)];
             const int valid = min(BLK, p.N - j * BLK);
             ok = mbar_wait_warp(bar(L::B_SF + (t & 1)), (t >> 1) & 1, ctl);
             if (!ok) break;
             tc_fence_after();
             float s[BLK];
             {
-                uint32_t raw[32];
+                uint32_t raw[BLK];
+                if constexpr (BLK == 128) {
+                    tmem_ld128_wait(tmem + lane_base + (t & 1) * 128, raw);
+                } else {
 #pragma unroll
-                for (int c = 0; c < BLK / 32; ++c) {
-                    tmem_ld32(tmem + lane_base + (t & 1) * 128 + c * 32, raw);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) s[c * 32 + e] = __uint_as_float(raw[e]);
+                    for (int c = 0; c < BLK / 32; ++c) tmem_ld32_wait(tmem + lane_base + (t & 1) * 128 + c * 32, raw + c * 32);
                 }
-            }
-            float mt = -INFINITY;
 #pragma unroll
-            for (int c = 0; c < BLK; ++c)
-                if (c < valid) mt = fmaxf(mt, s[c]);
-            const float mt2 = mt * p.scale_log2;
+                for (int c = 0; c < BLK; ++c) s[c] = __uint_as_float(raw[c]);
+            }
+            if (valid < BLK) {                      // ragged last key block only
+#pragma unroll
+                for (int c = 0; c < BLK; ++c)
+                    if (c >= valid) s[c] = -INFINITY;
+            }
+            // row max: four independent three-input chains
+            float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
+#pragma unroll
+            for (int c = 4; c < BLK; c += 8) {
+                mx0 = fmax3(mx0, s[c], s[c + 4]);
+                mx1 = fmax3(mx1, s[c + 1], s[c + 5]);
+                mx2 = fmax3(mx2, s[c + 2], s[c + 6]);
+                mx3 = fmax3(mx3, s[c + 3], s[c + 7]);
+            }
+            const float mt2 = fmax3(mx0, mx1, fmaxf(mx2, mx3)) * sc;
             const bool upd = mt2 > m_run + kRescaleLog2;
             const float m_new = upd ? mt2 : m_run;
             const float alpha = upd ? ex2_approx(m_run - m_new) : 1.f;
-            // P enters the PV MMA as bf16; O is normalised by the sum of those rounded
-            // weights (lq), so O stays an exact convex combination of the weights used.
-            // The unrounded sum (l) gives the LSE output.
-            float sum = 0.f, sumq = 0.f;
+            // P = 2^(s*scale_log2 - m): packed FMA, MUFU exp2, bf16 pack
             uint32_t pk[BLK / 2];
+            float ls0 = 0.f, ls1 = 0.f, ls2 = 0.f, ls3 = 0.f;
 #pragma unroll
             for (int c = 0; c < BLK; c += 2) {
-                const float p0 = (c < valid) ? ex2_approx(fmaf(s[c], p.scale_log2, -m_new)) : 0.f;
-                const float p1 = (c + 1 < valid) ? ex2_approx(fmaf(s[c + 1], p.scale_log2, -m_new)) : 0.f;
-                sum += p0 + p1;
-                const uint32_t w = pack_bf16x2(p0, p1);
-                sumq += __uint_as_float(w << 16) + __uint_as_float(w & 0xFFFF0000u);
-                pk[c / 2] = w;
+                float x0, x1;
+                ffma2(x0, x1, s[c], s[c + 1], sc, sc, -m_new, -m_new);
+                const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+                pk[c / 2] = pack_bf16x2(p0, p1);
+                if constexpr (WITH_LSE) {
+                    if ((c & 2) == 0) fadd2(ls0, ls1, ls0, ls1, p0, p1);
+                    else fadd2(ls2, ls3, ls2, ls3, p0, p1);
+                }
             }
-            l_run = l_run * alpha + sum;
-            lq_run = lq_run * alpha + sumq;
+            if constexpr (WITH_LSE) l_run = l_run * alpha + ((ls0 + ls1) + (ls2 + ls3));
             m_run = m_new;
 #pragma unroll
-            for (int c = 0; c < BLK / 32; ++c)
-                tmem_st16(tmem + lane_base + (t & 1) * 128 + c * 16, pk + c * 16);
-            if (__any_sync(0xffffffffu, upd && t > 0)) {
-                // O accumulated through PV_{t-1}: wait for it, then rescale rows in place.
+            for (int c = 0; c < BLK / 32; ++c) tmem_st16(tmem + lane_base + (t & 1) * 128 + c * 16, pk + c * 16);
+            // Consume the completion of PV_{t-1} on every tile.  An mbarrier parity wait is
+            // only unambiguous while the waiter is at most one phase behind; waiting on
+            // every phase keeps it so (PV_t cannot start before this tile's P is ready), and
+            // by now PV_{t-1}, issued before this tile's softmax began, has normally finished.
+            if (t > 0) {
                 ok = mbar_wait_warp(bar(L::B_O), (t - 1) & 1, ctl);
                 if (!ok) break;
+            }
+            if (__any_sync(0xffffffffu, upd && t > 0)) {
+                // rescale [O | rowsum], accumulated through PV_{t-1}, in place
                 tc_fence_after();
                 const float a_row = (upd && t > 0) ? alpha : 1.f;
                 uint32_t raw[32];
 #pragma unroll
-                for (int c = 0; c < D / 32; ++c) {
-                    tmem_ld32(tmem + lane_base + 256 + c * 32, raw);
-                    tmem_wait_ld();
+                for (int c = 0; c < (NPV + 31) / 32; ++c) {
+                    tmem_ld32_wait(tmem + lane_base + kTmemO + c * 32, raw);
 #pragma unroll
                     for (int e = 0; e < 32; ++e) raw[e] = __float_as_uint(__uint_as_float(raw[e]) * a_row);
-                    tmem_st32(tmem + lane_base + 256 + c * 32, raw);
+                    tmem_st32(tmem + lane_base + kTmemO + c * 32, raw);
                 }
             }
             tmem_wait_st();
@@ -339,35 +393,45 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         // ---- epilogue ----
         if (__all_sync(0xffffffffu, ok && !*abort_flag)) {
             const bool row_ok = r < BLK && (i * BLK + r) < Nq;
+            // completion of the last PV (the loop consumed every earlier one)
             if (nkept > 0) ok = mbar_wait_warp(bar(L::B_O), (nkept - 1) & 1, ctl);
             if (ok) {
                 tc_fence_after();
-                const float inv_l = nkept > 0 ? 1.f / lq_run : 0.f;
-                const float lse_val = nkept > 0 ? (m_run + lg2_approx(l_run)) * 0.69314718055994530942f : -INFINITY;
+                float lsum = 0.f;
+                if (nkept > 0) {
+                    uint32_t raw[32];
+                    tmem_ld32_wait(tmem + lane_base + kTmemO + D, raw);
+                    lsum = __uint_as_float(raw[0]);
+                }
+                const float inv_l = nkept > 0 ? 1.f / lsum : 0.f;
+                float lse_val = -INFINITY;
+                if constexpr (WITH_LSE) {
+                    if (nkept > 0) lse_val = (m_run + lg2_approx(l_run)) * 0.69314718055994530942f;
+                }
                 // destination rows: the row itself, or every token an anchor stands for
                 int tok0 = 0, ncopy = 0, copy_stride = 0;
                 if (row_ok) {
                     const int a = i * BLK + r;
                     if (!rep) {
-                        tok0 = a; ncopy = 1;
+                        tok0 = a;
+                        ncopy = 1;
                     } else {
                         const int nva = p.F * p.Ar * p.Wl;
+                        tok0 = anchor_token(p, a);
                         if (a < nva) {
-                            tok0 = anchor_token(p, a);
                             const int ya = (a / p.Wl) % p.Ar;
                             ncopy = min(p.stride, p.Hl - ya * p.stride);
                             copy_stride = p.Wl;
                         } else {
-                            tok0 = anchor_token(p, a); ncopy = 1;
+                            ncopy = 1;
                         }
                     }
                 }
-                uint32_t raw[32];
 #pragma unroll
                 for (int c = 0; c < D / 32; ++c) {
+                    uint32_t raw[32];
                     if (nkept > 0) {
-                        tmem_ld32(tmem + lane_base + 256 + c * 32, raw);
-                        tmem_wait_ld();
+                        tmem_ld32_wait(tmem + lane_base + kTmemO + c * 32, raw);
                     } else {
 #pragma unroll
                         for (int e = 0; e < 32; ++e) raw[e] = 0u;
@@ -377,11 +441,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         for (int e = 0; e < 32; ++e) raw[e] = __float_as_uint(__uint_as_float(raw[e]) * inv_l);
                         for (int cp = 0; cp < ncopy; ++cp) {
                             const size_t tok = static_cast<size_t>(tok0 + cp * copy_stride);
-                            uint4* d = reinterpret_cast<uint4*>(reinterpret_cast<float*>(p.o) +
-                                                                (static_cast<size_t>(h) * p.N + tok) * D + c * 32);
-#pragma unroll
-                            for (int v4 = 0; v4 < 8; ++v4)
-                                d[v4] = make_uint4(raw[4 * v4], raw[4 * v4 + 1], raw[4 * v4 + 2], raw[4 * v4 + 3]);
+                            store_row32_f32(reinterpret_cast<float*>(p.o) + (static_cast<size_t>(h) * p.N + tok) * D +
+                                                c * 32, raw);
                         }
                     } else {
                         uint32_t packed[16];
@@ -391,7 +452,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                                                     __uint_as_float(raw[2 * e + 1]) * inv_l);
                         for (int cp = 0; cp < ncopy; ++cp) {
                             const size_t tok = static_cast<size_t>(tok0 + cp * copy_stride);
-                            store_row_chunk(p.o + (static_cast<size_t>(h) * p.N + tok) * D + c * 32, packed);
+                            store_row32_bf16(p.o + (static_cast<size_t>(h) * p.N + tok) * D + c * 32, packed);
                         }
                     }
                 }

@@ -173,8 +173,7 @@ block_energy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 uint32_t raw[32];
 #pragma unroll
                 for (int c = 0; c < BLK / 32; ++c) {
-                    tmem_ld32(tmem + lane_base + b * 128 + c * 32, raw);
-                    tmem_wait_ld();
+                    tmem_ld32_wait(tmem + lane_base + b * 128 + c * 32, raw);
 #pragma unroll
                     for (int e = 0; e < 32; ++e) s[c * 32 + e] = __uint_as_float(raw[e]);
                 }

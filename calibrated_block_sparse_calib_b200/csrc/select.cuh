@@ -233,16 +233,20 @@ csr_fill_kernel(const uint8_t* __restrict__ mask, int rows, int nk, const int32_
     }
 }
 
-// Longest-first schedule, one block of 1024 threads: a counting sort of the rows by
-// kept count (descending), stable in row index.  Shared memory: histogram of 32768 bins.
+// Schedule: heads in order (so the K/V working set of the CTAs in flight is one or two
+// heads and stays in L2), and within a head the query blocks longest-first.  One block of
+// 1024 threads per head: a counting sort of the head's rows by kept count (descending),
+// stable in row index.  Shared memory: a histogram of 32768 bins.
 constexpr int kSchedBins = 32768;
 __global__ void __launch_bounds__(1024)
-schedule_kernel(const int32_t* __restrict__ row_ptr, int rows, int nq, int32_t* __restrict__ work) {
+schedule_kernel(const int32_t* __restrict__ row_ptr, int nq, int32_t* __restrict__ work) {
     extern __shared__ int32_t hist[];                // [kSchedBins]
     const int tid = threadIdx.x, nt = blockDim.x;
+    const int h = blockIdx.x;
+    const int r0 = h * nq;
     for (int b = tid; b < kSchedBins; b += nt) hist[b] = 0;
     __syncthreads();
-    for (int r = tid; r < rows; r += nt) {
+    for (int r = r0 + tid; r < r0 + nq; r += nt) {
         const int c = min(row_ptr[r + 1] - row_ptr[r], kSchedBins - 1);
         atomicAdd(&hist[kSchedBins - 1 - c], 1);     // bin order = count descending
     }
@@ -272,9 +276,10 @@ schedule_kernel(const int32_t* __restrict__ row_ptr, int rows, int nq, int32_t* 
     // stable scatter by one warp, rows in index order
     if (tid < 32) {
         const uint32_t lane = lane_id();
-        for (int r0 = 0; r0 < rows; r0 += 32) {
-            const int r = r0 + static_cast<int>(lane);
-            const bool live = r < rows;
+        for (int i0 = 0; i0 < nq; i0 += 32) {
+            const int i = i0 + static_cast<int>(lane);
+            const bool live = i < nq;
+            const int r = r0 + i;
             const int bin = live ? kSchedBins - 1 - min(row_ptr[r + 1] - row_ptr[r], kSchedBins - 1) : -1;
             const uint32_t peers = __match_any_sync(0xffffffffu, bin);
             const int leader = __ffs(peers) - 1;
@@ -284,10 +289,7 @@ schedule_kernel(const int32_t* __restrict__ row_ptr, int rows, int nq, int32_t* 
                 hist[bin] = basepos + __popc(peers);
             }
             basepos = __shfl_sync(0xffffffffu, basepos, leader);
-            if (live) {
-                const int pos = basepos + __popc(peers & lanemask_lt());
-                work[pos] = ((r / nq) << 16) | (r % nq);
-            }
+            if (live) work[r0 + basepos + __popc(peers & lanemask_lt())] = (h << 16) | i;
             __syncwarp();
         }
     }

@@ -181,7 +181,7 @@ def mask_to_csr(mask: torch.Tensor):
 
 
 def build_schedule(row_ptr: torch.Tensor, H: int, nq: int) -> torch.Tensor:
-    """int32 work list (h << 16 | i), kept count descending, ties by (h, i)."""
+    """int32 work list (h << 16 | i): heads in order, longest rows first within a head."""
     _need(row_ptr, "row_ptr", torch.int32, (H * nq + 1,))
     work = torch.empty(H * nq, dtype=torch.int32, device=row_ptr.device)
     _check("calib_build_schedule", lib().calib_build_schedule(_ptr(row_ptr), H, nq, _ptr(work), _stream()))

@@ -126,9 +126,11 @@ calib_status calib_aggregate_masks(const int32_t* counts, int H, int nq, int nk,
 calib_status calib_mask_to_csr(const uint8_t* mask, int H, int nq, int nk,
                                int32_t* row_ptr_out, int16_t* col_idx_out, void* stream);
 
-/* Load-balancing order ([AdaSpa] §2 balances kernel load across heads of different
- * sparsity): work_out int32 [H*nq] = every row h << 16 | i, kept count descending, ties
- * by (h, i) ascending.  H, nq < 65536. */
+/* Processing order ([AdaSpa] §2 balances kernel load across heads of different
+ * sparsity): work_out int32 [H*nq] = every row h << 16 | i, heads ascending and, within
+ * a head, kept count descending (longest first), ties by i ascending.  Head-major order
+ * keeps the K/V blocks read by concurrently running tiles within one or two heads, so
+ * they stay in L2.  H < 32768, nq < 65536. */
 calib_status calib_build_schedule(const int32_t* row_ptr, int H, int nq,
                                   int32_t* work_out, void* stream);
 

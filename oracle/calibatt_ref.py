@@ -217,14 +217,17 @@ def mask_to_csr(mask: np.ndarray):
 
 
 def build_schedule(row_ptr: np.ndarray, H: int, nq: int) -> np.ndarray:
-    """Work list for load balancing by kept-block count: every (h, i) ordered by kept
-    count descending, ties by (h, i) ascending; entry = h << 16 | i.
+    """Work list for load balancing by kept-block count: heads in ascending order and,
+    within a head, query blocks by kept count descending (ties by query block
+    ascending); entry = h << 16 | i.
 
     [AdaSpa] §2 motivates balancing the kernel's load across heads of different
-    sparsity; longest-first order is the classic greedy for that."""
+    sparsity; longest-first order is the classic greedy for that.  Reading: the order is
+    head-major so that the key/value blocks the concurrently running tiles read belong to
+    one or two heads at a time (a locality choice; the pages fix no order)."""
     rp = np.asarray(row_ptr, np.int64)
     cnt = rp[1:] - rp[:-1]
-    order = sorted(range(H * nq), key=lambda r: (-int(cnt[r]), r))
+    order = sorted(range(H * nq), key=lambda r: (r // nq, -int(cnt[r]), r))
     return np.array([((r // nq) << 16) | (r % nq) for r in order], np.int32)
 
 

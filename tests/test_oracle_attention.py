@@ -169,8 +169,9 @@ def test_csr_round_trip_and_schedule_order():
     rows = (w >> 16) * nq + (w & 0xFFFF)
     assert sorted(rows.tolist()) == list(range(H * nq))
     cnt = np.diff(rp)[rows]
-    # count descending; within equal counts, row index ascending (independent check
-    # with numpy's lexsort)
-    ref = np.lexsort((np.arange(H * nq), -np.diff(rp)))
+    # heads in order; inside a head count descending, then row index ascending
+    # (independent check with numpy's lexsort)
+    ref = np.lexsort((np.arange(H * nq), -np.diff(rp), np.arange(H * nq) // nq))
     np.testing.assert_array_equal(rows, ref)
-    assert np.all(np.diff(cnt) <= 0)
+    for h in range(H):
+        assert np.all(np.diff(cnt[h * nq:(h + 1) * nq]) <= 0)
