@@ -100,6 +100,7 @@ calib_status launch_attn(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
                          const calib::AttnParams& p, int grid, cudaStream_t st) {
     constexpr int KST = 2, VST = 2;
     using L = calib::AttnSmem<D, BLK, KST, VST>;
+    static_assert(L::BYTES <= 232448, "shared memory budget");
     auto* fn = calib::attn_fwd_kernel<D, BLK, KST, VST, WITH_LSE>;
     if (calib_status s = ensure_smem(reinterpret_cast<const void*>(fn), L::BYTES)) return s;
     fn<<<grid, calib::kAttnThreads, L::BYTES, st>>>(tq, tk, tv, p);
@@ -168,7 +169,7 @@ calib_status launch_energy(const CUtensorMap& tq, const CUtensorMap& tk, const c
     using L = calib::EnergySmem<D, BLK, KST>;
     auto* fn = calib::block_energy_kernel<D, BLK, KST>;
     if (calib_status s = ensure_smem(reinterpret_cast<const void*>(fn), L::BYTES)) return s;
-    fn<<<grid, calib::kAttnThreads, L::BYTES, st>>>(tq, tk, p);
+    fn<<<grid, calib::kEnergyThreads, L::BYTES, st>>>(tq, tk, p);
     return launch_status();
 }
 
@@ -195,6 +196,7 @@ calib_status calib_device_check(void* stream) {
     if (cudaMemcpyFromSymbol(&v, calib::g_status, sizeof(v)) != cudaSuccess) return CALIB_ERR_CUDA;
     if (v && cudaMemcpyToSymbol(calib::g_status, &zero, sizeof(zero)) != cudaSuccess) return CALIB_ERR_CUDA;
     if (v & calib::STATUS_TIMEOUT) return CALIB_ERR_TIMEOUT;
+    if (v & calib::STATUS_SMEM_ALIGN) return CALIB_ERR_CUDA;
     if (v & calib::STATUS_BAD_ENERGY) return CALIB_ERR_INVALID;
     return CALIB_OK;
 }

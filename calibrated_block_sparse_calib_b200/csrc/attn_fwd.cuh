@@ -211,33 +211,39 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     for (int s = 0; s < VST; ++s) armed_v[s] = 0;
 
     if (warp == 0) {
-        // ===================== TMA producer =====================
-        if (lane == 0 && nkept > 0) {
+        // ===================== TMA producer (converged warp, one elected lane issues) ====
+        if (nkept > 0) {
             if (!rep) {
-                mbar_arrive_expect_tx(bar(L::B_Q), L::Q_BYTES);
-                for (int c = 0; c < CH; ++c)
-                    tma_load_3d(smem_u32(sQ + c * kTileM * 128), &tm_q, bar(L::B_Q), c * 64, i * BLK, h);
+                if (elect_one()) {
+                    mbar_arrive_expect_tx(bar(L::B_Q), L::Q_BYTES);
+                    for (int c = 0; c < CH; ++c)
+                        tma_load_3d(smem_u32(sQ + c * kTileM * 128), &tm_q, bar(L::B_Q), c * 64, i * BLK, h);
+                }
                 armed_q = 1;
             }
             auto issue_k = [&](int t) -> bool {
                 const int s = t % KST;
-                if (!mbar_wait(bar(L::B_KE + s), ((t / KST) & 1) ^ 1, ctl)) return false;
+                if (!mbar_wait_warp(bar(L::B_KE + s), ((t / KST) & 1) ^ 1, ctl)) return false;
                 const int j = p.col_idx[kidx(t)];
-                mbar_arrive_expect_tx(bar(L::B_KF + s), L::K_BYTES);
-                for (int c = 0; c < CH; ++c)
-                    tma_load_3d(smem_u32(sK + s * L::K_BYTES + c * L::CHUNK), &tm_k, bar(L::B_KF + s), c * 64,
-                                j * BLK, h);
+                if (elect_one()) {
+                    mbar_arrive_expect_tx(bar(L::B_KF + s), L::K_BYTES);
+                    for (int c = 0; c < CH; ++c)
+                        tma_load_3d(smem_u32(sK + s * L::K_BYTES + c * L::CHUNK), &tm_k, bar(L::B_KF + s), c * 64,
+                                    j * BLK, h);
+                }
                 ++armed_k[s];
                 return true;
             };
             auto issue_v = [&](int t) -> bool {
                 const int s = t % VST;
-                if (!mbar_wait(bar(L::B_VE + s), ((t / VST) & 1) ^ 1, ctl)) return false;
+                if (!mbar_wait_warp(bar(L::B_VE + s), ((t / VST) & 1) ^ 1, ctl)) return false;
                 const int j = p.col_idx[kidx(t)];
-                mbar_arrive_expect_tx(bar(L::B_VF + s), L::K_BYTES);
-                for (int c = 0; c < CH; ++c)
-                    tma_load_3d(smem_u32(sV + s * L::V_STAGE + c * L::CHUNK), &tm_v, bar(L::B_VF + s), c * 64,
-                                j * BLK, h);
+                if (elect_one()) {
+                    mbar_arrive_expect_tx(bar(L::B_VF + s), L::K_BYTES);
+                    for (int c = 0; c < CH; ++c)
+                        tma_load_3d(smem_u32(sV + s * L::V_STAGE + c * L::CHUNK), &tm_v, bar(L::B_VF + s), c * 64,
+                                    j * BLK, h);
+                }
                 ++armed_v[s];
                 return true;
             };
@@ -248,51 +254,57 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
         }
     } else if (warp == 1) {
-        // ===================== MMA issuer =====================
-        if (lane == 0 && nkept > 0) {
+        // ===================== MMA issuer (converged warp, one elected lane issues) ======
+        if (nkept > 0) {
             constexpr uint32_t idesc_qk = idesc_bf16_f32(kTileM, BLK, false, false);
             constexpr uint32_t idesc_pv = idesc_bf16_f32(kTileM, NPV, false, true);
             const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV);
-            bool ok = mbar_wait(bar(L::B_Q), 0, ctl);
+            bool ok = mbar_wait_warp(bar(L::B_Q), 0, ctl);
             tc_fence_after();
             auto issue_qk = [&](int t) -> bool {
                 const int s = t % KST;
-                if (!mbar_wait(bar(L::B_KF + s), (t / KST) & 1, ctl)) return false;
+                if (!mbar_wait_warp(bar(L::B_KF + s), (t / KST) & 1, ctl)) return false;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem + (t & 1) * 128;
+                if (elect_one()) {
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t inner = (kk & 3) * 32;   // K step of 16 bf16 inside a 128-B atom
-                    const uint64_t ad = smem_desc_sw128(sQa + (kk >> 2) * kTileM * 128 + inner, 16, 1024);
-                    const uint64_t bd =
-                        smem_desc_sw128(sKa + s * L::K_BYTES + (kk >> 2) * L::CHUNK + inner, 16, 1024);
-                    umma_ss(d_tmem, ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t inner = (kk & 3) * 32;   // K step of 16 bf16 inside a 128-B atom
+                        const uint64_t ad = smem_desc_sw128(sQa + (kk >> 2) * kTileM * 128 + inner, 16, 1024);
+                        const uint64_t bd =
+                            smem_desc_sw128(sKa + s * L::K_BYTES + (kk >> 2) * L::CHUNK + inner, 16, 1024);
+                        umma_ss(d_tmem, ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
+                    }
+                    umma_commit(bar(L::B_SF + (t & 1)));
+                    umma_commit(bar(L::B_KE + s));
                 }
-                umma_commit(bar(L::B_SF + (t & 1)));
-                umma_commit(bar(L::B_KE + s));
+                __syncwarp();
                 return true;
             };
             if (ok) ok = issue_qk(0);
             for (int t = 0; ok && t < nkept; ++t) {
                 if (t + 1 < nkept) {
                     // S buffer (t+1)&1 last held P_{t-1}: PV_{t-1} must be complete.
-                    if (t >= 1) ok = mbar_wait(bar(L::B_O), (t - 1) & 1, ctl);
+                    if (t >= 1) ok = mbar_wait_warp(bar(L::B_O), (t - 1) & 1, ctl);
                     if (ok) ok = issue_qk(t + 1);
                     if (!ok) break;
                 }
                 const int sv = t % VST;
-                ok = mbar_wait(bar(L::B_PF + (t & 1)), (t >> 1) & 1, ctl);
-                if (ok) ok = mbar_wait(bar(L::B_VF + sv), (t / VST) & 1, ctl);
+                ok = mbar_wait_warp(bar(L::B_PF + (t & 1)), (t >> 1) & 1, ctl);
+                if (ok) ok = mbar_wait_warp(bar(L::B_VF + sv), (t / VST) & 1, ctl);
                 if (!ok) break;
                 tc_fence_after();
                 const uint32_t a_tmem = tmem + (t & 1) * 128;
+                if (elect_one()) {
 #pragma unroll
-                for (int kk = 0; kk < BLK / 16; ++kk) {
-                    const uint64_t bd = smem_desc_sw128(sVa + sv * L::V_STAGE + kk * 16 * 128, L::CHUNK, 1024);
-                    umma_ts(tmem + kTmemO, a_tmem + kk * 8, bd, idesc_pv, (t > 0 || kk > 0) ? 1u : 0u);
+                    for (int kk = 0; kk < BLK / 16; ++kk) {
+                        const uint64_t bd = smem_desc_sw128(sVa + sv * L::V_STAGE + kk * 16 * 128, L::CHUNK, 1024);
+                        umma_ts(tmem + kTmemO, a_tmem + kk * 8, bd, idesc_pv, (t > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    umma_commit(bar(L::B_O));
+                    umma_commit(bar(L::B_VE + sv));
                 }
-                umma_commit(bar(L::B_O));
-                umma_commit(bar(L::B_VE + sv));
+                __syncwarp();
             }
         }
     } else {
@@ -334,15 +346,20 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 for (int c = 0; c < BLK; ++c)
                     if (c >= valid) s[c] = -INFINITY;
             }
-            // row max: four independent three-input chains
+            // row max: four independent three-input chains over s[4 .. BLK-5], then the
+            // last four columns
             float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
 #pragma unroll
-            for (int c = 4; c < BLK; c += 8) {
+            for (int c = 4; c + 8 <= BLK; c += 8) {
                 mx0 = fmax3(mx0, s[c], s[c + 4]);
                 mx1 = fmax3(mx1, s[c + 1], s[c + 5]);
                 mx2 = fmax3(mx2, s[c + 2], s[c + 6]);
                 mx3 = fmax3(mx3, s[c + 3], s[c + 7]);
             }
+            mx0 = fmaxf(mx0, s[BLK - 4]);
+            mx1 = fmaxf(mx1, s[BLK - 3]);
+            mx2 = fmaxf(mx2, s[BLK - 2]);
+            mx3 = fmaxf(mx3, s[BLK - 1]);
             const float mt2 = fmax3(mx0, mx1, fmaxf(mx2, mx3)) * sc;
             const bool upd = mt2 > m_run + kRescaleLog2;
             const float m_new = upd ? mt2 : m_run;

@@ -24,6 +24,7 @@
 namespace calib {
 
 constexpr uint32_t kEnergyTmemCols = 256;
+constexpr int kEnergyThreads = 192;
 
 struct EnergyParams {
     const __nv_bfloat16* q;   // [H, N, D] (read directly only for gathered rows)
@@ -53,7 +54,7 @@ struct EnergySmem {
 };
 
 template <int D, int BLK, int KST>
-__global__ void __launch_bounds__(kAttnThreads, 1)
+__global__ void __launch_bounds__(kEnergyThreads, 1)
 block_energy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const EnergyParams p) {
     using L = EnergySmem<D, BLK, KST>;

@@ -73,7 +73,8 @@ const char* calib_status_string(calib_status s);
 /* Synchronises `stream`, then reads and clears the status word of the current device.
  * Returns CALIB_ERR_TIMEOUT if any kernel since the last check gave up on a bounded
  * wait, CALIB_ERR_INVALID if a selection kernel met a negative or non-finite energy
- * (treated as 0), CALIB_ERR_CUDA on a CUDA error, else CALIB_OK. */
+ * (treated as 0), CALIB_ERR_CUDA on a CUDA error (or a kernel that found its shared
+ * memory misaligned and did nothing), else CALIB_OK. */
 calib_status calib_device_check(void* stream);
 
 /* Row log-sum-exp and block energies, fused ([zh] §2.2A, [de] §2A.1, [fr] §2.B.1: split
