@@ -18,6 +18,7 @@ host cores.  `--impl reference` times that oracle alone as the reference arm.
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import math
 import os
@@ -34,6 +35,17 @@ if ROOT not in sys.path:
 
 METRIC = "sparse attn TFLOPS (kept-only & dense-equiv) + % BF16 TC peak at 30% density"
 UNIT = "TFLOPS"
+
+# DRAM bytes (read + write) of one attn_fwd_kernel launch on the wan13b workload, from an
+# ncu capture (profiles/attn_fwd_wan13b.md), valid only for the kernel sources it was taken
+# on: reported as roofline.traffic while the source hashes still match, else null.
+NCU_TRAFFIC = {("wan13b", "70b321627e5a", "e4390e39220d"): 302_647_040 + 86_838_016}
+
+
+def _src_sha(name):
+    path = os.path.join(ROOT, "calibrated_block_sparse_calib_b200", "csrc", name)
+    with open(path, "rb") as f:
+        return hashlib.sha1(f.read()).hexdigest()[:12]
 
 
 def _peaks():
@@ -180,6 +192,7 @@ def main():
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="wan13b", choices=["wan13b", "wan14b720p", "mochi1"])
+    ap.add_argument("--timestep", type=int, default=0, help="timestep of the mask schedule (mochi1)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true", help="skip dense / e2e / calibration legs")
@@ -207,7 +220,7 @@ def main():
     s = wl.shape
     B, D, N, H = s.block, s.D, s.N, s.H
     q, k, v = synth.make_qkv(wl, device=dev)
-    mask_np = synth.make_head_masks(wl)
+    mask_np = synth.make_head_masks(wl, timestep=args.timestep)
     mask = torch.from_numpy(mask_np).to(dev)
     bl = ops.BlockList.from_mask(mask, B)
     rep = [h in wl.repeat_heads for h in range(H)]
@@ -259,6 +272,24 @@ def main():
         ms_dense = _time_calls(lambda: ops.sparse_attn_fwd(q, k, v, bl_dense, out=out), 10, 3, torch)
         extras["dense_kernel"] = {"ms": ms_dense, "tflops": flops_dense / (ms_dense * 1e-3) / 1e12,
                                   "speedup_sparse_vs_dense": ms_dense / ms}
+        # density sweep on the same shapes (seeded generator masks), against the dense kernel
+        if wl.name == "wan13b" and not any(rep):
+            sweep = {}
+            for d in (0.10, 0.20, 0.30, 0.50):
+                m_d = synth.make_head_masks(wl, density=d)
+                bl_d = ops.BlockList.from_mask(torch.from_numpy(m_d).to(dev), B)
+                fk = kept_flops(m_d, N, D, B)
+                ms_d = _time_calls(lambda: ops.sparse_attn_fwd(q, k, v, bl_d, out=out), 20, 3, torch)
+                sweep[f"{d:.2f}"] = {"density": round(fk / flops_dense, 4), "ms": ms_d,
+                                     "kept_tflops": fk / (ms_d * 1e-3) / 1e12,
+                                     "dense_equiv_tflops": flops_dense / (ms_d * 1e-3) / 1e12,
+                                     "frac_of_bf16_peak": fk / (ms_d * 1e-3) / 1e12 / peaks["bf16_tflops"],
+                                     "speedup_vs_dense": ms_dense / ms_d}
+            sweep["1.00"] = {"density": 1.0, "ms": ms_dense, "kept_tflops": flops_dense / (ms_dense * 1e-3) / 1e12,
+                             "dense_equiv_tflops": flops_dense / (ms_dense * 1e-3) / 1e12,
+                             "frac_of_bf16_peak": flops_dense / (ms_dense * 1e-3) / 1e12 / peaks["bf16_tflops"],
+                             "speedup_vs_dense": 1.0}
+            extras["density_sweep"] = sweep
         # end to end through the public API with host buffers
         qh, kh, vh = (t.cpu().pin_memory() for t in (q, k, v))
         oh = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
@@ -308,8 +339,10 @@ def main():
         "dense_equiv_tflops": flops_dense * world / (ms * 1e-3) / 1e12,
         "frac_of_bf16_peak": value / world / peaks["bf16_tflops"],
         "roofline": {"bound": "tensor", "achieved": value / world, "peak": peaks["bf16_tflops"],
-                     "unit": "TFLOP/s", "frac": value / world / peaks["bf16_tflops"], "traffic": None,
-                     "peak_source": f"{peaks['source']} bf16 burst", "kernel": "attn_fwd_kernel<128,128,2,2>",
+                     "unit": "TFLOP/s", "frac": value / world / peaks["bf16_tflops"],
+                     "traffic": NCU_TRAFFIC.get((wl.name, _src_sha("attn_fwd.cuh"), _src_sha("ptx.cuh"))),
+                     "algorithmic_bytes": 4 * q.numel() * q.element_size(),
+                     "peak_source": f"{peaks['source']} bf16 burst", "kernel": f"attn_fwd_kernel<{D},{B},2,2,0>",
                      "frac_of_sustained": value / world / peaks["bf16_tflops_sustained"]},
         "gpu_launches": args.steps,
         "clocks": clk.summary(),

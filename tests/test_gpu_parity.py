@@ -410,3 +410,63 @@ def test_wait_timeout_selftest_keeps_context_usable(tiny_inputs):
     e = ops.block_energy(q.cuda(), k.cuda(), wl.shape.block)
     ops.device_check()
     assert torch.isfinite(e).all()
+
+
+def _sampled_rows(rng, nblk, block, N, k=4):
+    blocks = sorted(set(rng.choice(nblk - 1, size=k - 1, replace=False).tolist()) | {nblk - 1})
+    return blocks, np.concatenate([np.arange(i * block, min((i + 1) * block, N)) for i in blocks])
+
+
+def test_wan14b720p_repeat_heads_sampled():
+    # 40 heads x 75600 tokens; heads h % 4 == 3 use spatial repetition with stride 4 along
+    # latent rows (45 rows -> anchors 0, 4, ..., 44).  Checked: one plain head and one
+    # repeat head on sampled query blocks, plus every row of the repeat head equal to its
+    # anchor's row.
+    wl = synth.WORKLOADS["wan14b720p"]
+    s = wl.shape
+    q, k, v = synth.make_qkv(wl, device="cuda")
+    mask = synth.make_head_masks(wl)
+    rep = [h in wl.repeat_heads for h in range(s.H)]
+    bl = _blist(mask, s.block)
+    O = ops.sparse_attn_fwd_repeat(q, k, v, bl, rep, s.F, s.Hl, s.Wl, s.n_text, wl.repeat_stride)
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(21)
+    scale = 1 / math.sqrt(s.D)
+    # plain head 0
+    blocks, rows = _sampled_rows(rng, s.nblk, s.block, s.N)
+    qh, kh, vh = (to64(t[0:1]) for t in (q, k, v))
+    O_ref, _ = oracle.sparse_attention(qh, kh, vh, scale, s.block, mask[0:1], q_blocks=blocks)
+    check_attn(O[0:1], O_ref, rows=rows)
+    # repeat head 3: sampled anchor blocks, compared on the anchors' own token rows
+    h = 3
+    A = oracle.anchor_rows(s.F, s.Hl, s.Wl, s.n_text, wl.repeat_stride)
+    nqa = -(-len(A) // s.block)
+    ablocks = sorted(set(rng.choice(nqa - 1, size=3, replace=False).tolist()) | {nqa - 1})
+    qa = to64(q[h])[A][None]
+    kh, vh = to64(k[h:h + 1]), to64(v[h:h + 1])
+    Oa, _ = oracle.sparse_attention(qa, kh, vh, scale, s.block, mask[h:h + 1, :nqa], q_blocks=ablocks)
+    arows = np.concatenate([np.arange(i * s.block, min((i + 1) * s.block, len(A))) for i in ablocks])
+    check_attn(O[h][A][None], Oa, rows=arows)
+    Oc = O[h].cpu()
+    amap = np.array([oracle.anchor_index_of_token(t, s.F, s.Hl, s.Wl, s.n_text, wl.repeat_stride)
+                     for t in range(0, s.N, 997)])
+    for t, a in zip(range(0, s.N, 997), amap):
+        assert torch.equal(Oc[t], Oc[int(A[a])])
+
+
+def test_mochi1_text_tokens_sampled():
+    # 24 heads x (44520 video + 256 text) tokens, timestep 7 mask (~20% density) with every
+    # key block holding text and every query block holding text kept.
+    wl = synth.WORKLOADS["mochi1"]
+    s = wl.shape
+    q, k, v = synth.make_qkv(wl, device="cuda")
+    mask = synth.make_head_masks(wl, timestep=7)
+    bl = _blist(mask, s.block)
+    O = ops.sparse_attn_fwd(q, k, v, bl)
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(31)
+    blocks, rows = _sampled_rows(rng, s.nblk, s.block, s.N)
+    heads = [0, 23]
+    qh, kh, vh = (to64(t[heads]) for t in (q, k, v))
+    O_ref, _ = oracle.sparse_attention(qh, kh, vh, 1 / math.sqrt(s.D), s.block, mask[heads], q_blocks=blocks)
+    check_attn(O[heads], O_ref, rows=rows)
