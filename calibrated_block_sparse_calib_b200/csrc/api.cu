@@ -98,7 +98,11 @@ calib_status launch_status() {
 template <int D, int BLK, bool WITH_LSE>
 calib_status launch_attn(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                          const calib::AttnParams& p, int grid, cudaStream_t st) {
-    constexpr int KST = 2, VST = 2;
+#ifndef CALIB_ATTN_KST
+#define CALIB_ATTN_KST 3
+#define CALIB_ATTN_VST 3
+#endif
+    constexpr int KST = CALIB_ATTN_KST, VST = CALIB_ATTN_VST;
     using L = calib::AttnSmem<D, BLK, KST, VST>;
     static_assert(L::BYTES <= 232448, "shared memory budget");
     auto* fn = calib::attn_fwd_kernel<D, BLK, KST, VST, WITH_LSE>;

@@ -7,35 +7,43 @@
 // [fr] §2.C), and for spatial-repetition heads only on anchor rows whose output is
 // broadcast to the other rows of their frame ([zh] §2.2B, [fr] §2.C).
 //
-// One CTA per work item (head h, query block i).  192 threads:
+// One CTA per work item (head h, query block i).  320 threads:
 //   warp 0      TMA producer: Q tile once (repeat heads: nothing, their anchor rows are
 //               gathered by the softmax warps), then K_j / V_j for each kept j through
 //               KST / VST-deep rings (K runs one tile ahead of V).
-//   warp 1      TMEM owner (512 columns) and single-thread MMA issuer:
-//               S_t = Q K_j^T        SS MMA, M=128, N=B, K=D, into S buffer t%2;
-//               [O|l] += P_t [V_j|1] TS MMA, M=128, N=D+16, K=B: P from TMEM, V from SMEM.
-//               The 16 extra B columns are a constant all-ones chunk placed after each V
-//               stage, so column D of the accumulator is the row sum of the bf16 P that
-//               entered the product (the softmax normaliser, exactly consistent with O).
-//   warps 2..5  softmax + epilogue, one query row per thread (TMEM lane = row): online
-//               row max in the log2 domain with lazy rescaling (O is rescaled only when the
-//               max grows by more than 2^8), P = 2^(x - m) written back over S as bf16,
-//               final division by the accumulated row sum, bf16 (or fp32) stores.
+//   warp 1      TMEM owner (512 columns) and MMA issuer (one elected lane of the
+//               converged warp):
+//               S_t = Q K_j^T           SS MMA, M=128, N=B, K=D, into S buffer t%2;
+//               O_h += P_t,h V_j,h      TS MMA, M=128, N=D, K=B/2, for the two column
+//                                       halves h of the tile: P from TMEM, V from SMEM.
+//   warps 2..9  softmax + epilogue.  Each query row (TMEM lane) is split between two
+//               warps: warps 2..5 own the first half of every key tile's columns, warps
+//               6..9 the second half.  The two halves run INDEPENDENT online-softmax
+//               chains (own running max m_h, own row sum l_h, own accumulator O_h), so
+//               no per-tile exchange couples them; the epilogue merges them once:
+//               O = (O_0 2^(m_0-m) + O_1 2^(m_1-m)) / (l_0 2^(m_0-m) + l_1 2^(m_1-m)).
+//               Per tile a thread loads its B/2 logits, takes the row max in the log2
+//               domain with lazy rescaling (O_h is rescaled only when m_h grows by more
+//               than 2^8), writes P = 2^(x - m_h) back over its own S columns as bf16 and
+//               adds the bf16-ROUNDED P into l_h, so the normaliser is exactly the sum of
+//               the weights that entered the PV product.
 // Each row's key list is walked starting at its diagonal block (the first kept key block
 // at or after the query block), where local attention peaks, so the running max is
 // usually final after the first tile and O is rarely rescaled.
-// Tensor memory: S0 = cols [0,128), S1 = [128,256), [O|l] = [256, 256+D+16).
+// Tensor memory: S0 = cols [0,128), S1 = [128,256), O_0 = [256, 256+D), O_1 = [256+D, 256+2D).
 #pragma once
 #include <cuda_bf16.h>
 #include "ptx.cuh"
 
 namespace calib {
 
-constexpr int kAttnThreads = 192;
+constexpr int kAttnThreads = 320;
+constexpr int kSoftmaxThreads = 256;      // warps 2..9
 constexpr int kTileM = 128;               // query rows per tile (MMA M)
 constexpr float kRescaleLog2 = 8.0f;      // rescale O only when the row max grows by > 2^8
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kTmemO = 256;          // first column of the [O | rowsum] accumulator
+constexpr uint32_t kTmemO = 256;          // first column of O_0 (O_1 follows at kTmemO + D)
+constexpr uint32_t kBarSoftmax = 1;       // named barrier of the softmax warps
 
 struct AttnParams {
     const __nv_bfloat16* q;   // [H, N, D] (read directly only for repeat-head gathers)
@@ -100,15 +108,17 @@ struct AttnSmem {
     static constexpr uint32_t CHUNK = BLK * 128;          // one 64-column chunk of a K/V tile
     static constexpr uint32_t Q_BYTES = CH * kTileM * 128;
     static constexpr uint32_t K_BYTES = CH * CHUNK;
-    static constexpr uint32_t V_STAGE = (CH + 1) * CHUNK; // V chunks + the all-ones chunk
     static constexpr uint32_t OFF_K = Q_BYTES;
     static constexpr uint32_t OFF_V = OFF_K + KST * K_BYTES;
-    static constexpr uint32_t OFF_BAR = OFF_V + VST * V_STAGE;
+    static constexpr uint32_t OFF_BAR = OFF_V + VST * K_BYTES;
     // barrier indices
     static constexpr int B_Q = 0, B_KF = 1, B_KE = B_KF + KST, B_VF = B_KE + KST,
                          B_VE = B_VF + VST, B_SF = B_VE + VST, B_PF = B_SF + 2, B_O = B_PF + 2,
                          B_DRAIN = B_O + 1, NBARS = B_DRAIN + 1;
     static constexpr uint32_t OFF_MISC = OFF_BAR + NBARS * 8;   // tmem base, abort flag, t0
+    // The epilogue's exchange of (m, l) between the two halves of a row, float4 [2][128],
+    // reuses the Q tile: by then every MMA that read Q has completed.
+    static constexpr uint32_t OFF_XCH = 0;
     // + alignment slack; at least 120 KB so that one CTA (holding all 512 TMEM columns)
     // is resident per SM and no CTA waits in tcgen05.alloc.
     static constexpr uint32_t RAW = OFF_MISC + 16 + 1024;
@@ -121,7 +131,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
     using L = AttnSmem<D, BLK, KST, VST>;
     constexpr int CH = L::CH;
-    constexpr int NPV = D + 16;                            // PV MMA N: O columns + row sum
+    constexpr int HC = BLK / 2;                            // key columns per softmax half
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
@@ -158,7 +168,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         mbar_init(bar(L::B_Q), rep ? 128u : 1u);
         for (int s = 0; s < KST; ++s) { mbar_init(bar(L::B_KF + s), 1); mbar_init(bar(L::B_KE + s), 1); }
         for (int s = 0; s < VST; ++s) { mbar_init(bar(L::B_VF + s), 1); mbar_init(bar(L::B_VE + s), 1); }
-        for (int b = 0; b < 2; ++b) { mbar_init(bar(L::B_SF + b), 1); mbar_init(bar(L::B_PF + b), 128); }
+        for (int b = 0; b < 2; ++b) mbar_init(bar(L::B_SF + b), 1);
+        for (int b = 0; b < 2; ++b) mbar_init(bar(L::B_PF + b), kSoftmaxThreads);
         mbar_init(bar(L::B_O), 1);
         mbar_init(bar(L::B_DRAIN), 1);
         *abort_flag = 0;
@@ -179,17 +190,6 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     if (warp == 1) {
         tmem_alloc(smem_u32(tmem_slot), kTmemCols);
         tmem_relinquish();
-    }
-    if (warp >= 2) {
-        // all-ones chunk after every V stage: bf16 1.0 = 0x3F80 (the swizzle is
-        // irrelevant for a constant tile)
-        const uint4 ones = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
-        for (int s = 0; s < VST; ++s) {
-            uint4* dst = reinterpret_cast<uint4*>(sV + s * L::V_STAGE + CH * L::CHUNK);
-            for (int x = static_cast<int>(threadIdx.x) - 64; x < static_cast<int>(L::CHUNK / 16); x += 128)
-                dst[x] = ones;
-        }
-        fence_proxy_async_smem();
     }
     tc_fence_before();
     __syncthreads();
@@ -241,7 +241,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 if (elect_one()) {
                     mbar_arrive_expect_tx(bar(L::B_VF + s), L::K_BYTES);
                     for (int c = 0; c < CH; ++c)
-                        tma_load_3d(smem_u32(sV + s * L::V_STAGE + c * L::CHUNK), &tm_v, bar(L::B_VF + s), c * 64,
+                        tma_load_3d(smem_u32(sV + s * L::K_BYTES + c * L::CHUNK), &tm_v, bar(L::B_VF + s), c * 64,
                                     j * BLK, h);
                 }
                 ++armed_v[s];
@@ -257,62 +257,83 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         // ===================== MMA issuer (converged warp, one elected lane issues) ======
         if (nkept > 0) {
             constexpr uint32_t idesc_qk = idesc_bf16_f32(kTileM, BLK, false, false);
-            constexpr uint32_t idesc_pv = idesc_bf16_f32(kTileM, NPV, false, true);
+            constexpr uint32_t idesc_pv = idesc_bf16_f32(kTileM, D, false, true);
             const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV);
             bool ok = mbar_wait_warp(bar(L::B_Q), 0, ctl);
             tc_fence_after();
-            auto issue_qk = [&](int t) -> bool {
+            // Every tcgen05.mma blocks its issuer while the tensor pipe's short queue is
+            // full, so any time this warp spends between MMA batches leaves the pipe idle.
+            // The loop has two wait points per tile, both normally already satisfied: the
+            // K/V tiles (loaded ahead) before QK, and P before PV.  Each wait's first
+            // try_wait is issued before the preceding MMA batch, so its latency (an mbarrier
+            // round trip, ~100 cycles) overlaps that batch's issue.
+            auto qk = [&](int t) {
                 const int s = t % KST;
-                if (!mbar_wait_warp(bar(L::B_KF + s), (t / KST) & 1, ctl)) return false;
-                tc_fence_after();
                 const uint32_t d_tmem = tmem + (t & 1) * 128;
-                if (elect_one()) {
 #pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint32_t inner = (kk & 3) * 32;   // K step of 16 bf16 inside a 128-B atom
-                        const uint64_t ad = smem_desc_sw128(sQa + (kk >> 2) * kTileM * 128 + inner, 16, 1024);
-                        const uint64_t bd =
-                            smem_desc_sw128(sKa + s * L::K_BYTES + (kk >> 2) * L::CHUNK + inner, 16, 1024);
-                        umma_ss(d_tmem, ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
-                    }
-                    umma_commit(bar(L::B_SF + (t & 1)));
-                    umma_commit(bar(L::B_KE + s));
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t inner = (kk & 3) * 32;   // K step of 16 bf16 inside a 128-B atom
+                    const uint64_t ad = smem_desc_sw128(sQa + (kk >> 2) * kTileM * 128 + inner, 16, 1024);
+                    const uint64_t bd = smem_desc_sw128(sKa + s * L::K_BYTES + (kk >> 2) * L::CHUNK + inner, 16, 1024);
+                    umma_ss(d_tmem, ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
                 }
-                __syncwarp();
-                return true;
+                umma_commit(bar(L::B_SF + (t & 1)));
+                umma_commit(bar(L::B_KE + s));
             };
-            if (ok) ok = issue_qk(0);
+            auto kf = [&](int t) { return bar(L::B_KF + t % KST); };
+            auto kf_par = [&](int t) -> uint32_t { return (t / KST) & 1; };
+            auto vf = [&](int t) { return bar(L::B_VF + t % VST); };
+            auto vf_par = [&](int t) -> uint32_t { return (t / VST) & 1; };
+            if (ok) ok = mbar_wait_warp(kf(0), 0, ctl);
+            if (ok) {
+                tc_fence_after();
+                if (elect_one()) qk(0);
+            }
+            bool tok_k = nkept > 1 ? mbar_try_wait(kf(1), kf_par(1)) : true;
+            bool tok_v = mbar_try_wait(vf(0), vf_par(0));
             for (int t = 0; ok && t < nkept; ++t) {
-                if (t + 1 < nkept) {
-                    // S buffer (t+1)&1 last held P_{t-1}: PV_{t-1} must be complete.
-                    if (t >= 1) ok = mbar_wait_warp(bar(L::B_O), (t - 1) & 1, ctl);
-                    if (ok) ok = issue_qk(t + 1);
-                    if (!ok) break;
-                }
                 const int sv = t % VST;
-                ok = mbar_wait_warp(bar(L::B_PF + (t & 1)), (t >> 1) & 1, ctl);
-                if (ok) ok = mbar_wait_warp(bar(L::B_VF + sv), (t / VST) & 1, ctl);
+                if (t + 1 < nkept) ok = mbar_wait_warp_tok(kf(t + 1), kf_par(t + 1), tok_k, ctl);
+                if (ok) ok = mbar_wait_warp_tok(vf(t), vf_par(t), tok_v, ctl);
                 if (!ok) break;
                 tc_fence_after();
-                const uint32_t a_tmem = tmem + (t & 1) * 128;
+                const bool tok_p = mbar_try_wait(bar(L::B_PF + (t & 1)), (t >> 1) & 1);
+                // S buffer (t+1)&1 last held P_{t-1}, the A operand of PV_{t-1}.  This thread
+                // issued PV_{t-1} before this QK, and tcgen05.mma operations of one issuing
+                // thread execute in issue order, so QK_{t+1} overwrites the buffer only after
+                // PV_{t-1} has read it: no completion wait.
+                if (t + 1 < nkept && elect_one()) qk(t + 1);
+                ok = mbar_wait_warp_tok(bar(L::B_PF + (t & 1)), (t >> 1) & 1, tok_p, ctl);
+                if (!ok) break;
+                tc_fence_after();
+                tok_k = t + 2 < nkept ? mbar_try_wait(kf(t + 2), kf_par(t + 2)) : true;
+                tok_v = t + 1 < nkept ? mbar_try_wait(vf(t + 1), vf_par(t + 1)) : true;
                 if (elect_one()) {
+                    // O_h += P_t,h V_j,h for both column halves; P_t,h is packed bf16 in the
+                    // first HC/2 columns of the half's S columns
 #pragma unroll
-                    for (int kk = 0; kk < BLK / 16; ++kk) {
-                        const uint64_t bd = smem_desc_sw128(sVa + sv * L::V_STAGE + kk * 16 * 128, L::CHUNK, 1024);
-                        umma_ts(tmem + kTmemO, a_tmem + kk * 8, bd, idesc_pv, (t > 0 || kk > 0) ? 1u : 0u);
+                    for (int hf = 0; hf < 2; ++hf) {
+#pragma unroll
+                        for (int kk = 0; kk < HC / 16; ++kk) {
+                            const uint64_t bd =
+                                smem_desc_sw128(sVa + sv * L::K_BYTES + (hf * HC + kk * 16) * 128, L::CHUNK, 1024);
+                            umma_ts(tmem + kTmemO + hf * D, tmem + (t & 1) * 128 + hf * HC + kk * 8, bd, idesc_pv,
+                                    (t > 0 || kk > 0) ? 1u : 0u);
+                        }
                     }
                     umma_commit(bar(L::B_O));
                     umma_commit(bar(L::B_VE + sv));
                 }
-                __syncwarp();
             }
         }
     } else {
-        // ===================== softmax + epilogue (warps 2..5) =====================
+        // ===================== softmax + epilogue (warps 2..9) =====================
+        const int hf = static_cast<int>(warp - 2) >> 2;    // column half of every key tile
         const uint32_t q4 = warp & 3;
         const int r = static_cast<int>(q4 * 32 + lane);   // tile row == TMEM lane
         const uint32_t lane_base = (q4 * 32) << 16;
-        if (rep && nkept > 0) {
+        const uint32_t o_col = kTmemO + hf * D;            // this half's accumulator O_h
+        if (rep && nkept > 0 && hf == 0) {
             const int a = i * BLK + r;
             const __nv_bfloat16* src =
                 (a < Nq) ? p.q + (static_cast<size_t>(h) * p.N + anchor_token(p, a)) * D : nullptr;
@@ -321,162 +342,178 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             mbar_arrive(bar(L::B_Q));
         }
         const float sc = p.scale_log2;
-        float m_run = -INFINITY, l_run = 0.f;
+        float m_run = -INFINITY;   // running reference max of this half (log2 domain)
+        float l_run = 0.f;         // sum of the bf16-rounded P of this half
+        float l_ex = 0.f;          // exact fp32 sum (for the LSE output)
         bool ok = true;
         for (int t = 0; t < nkept; ++t) {
             const int j = p.col_idx[kidx(t)];
-            const int valid = min(BLK, p.N - j * BLK);
+            const int valid = min(BLK, p.N - j * BLK) - hf * HC;   // may be <= 0 (ragged tail)
             ok = mbar_wait_warp(bar(L::B_SF + (t & 1)), (t >> 1) & 1, ctl);
             if (!ok) break;
             tc_fence_after();
-            float s[BLK];
+            const uint32_t s_col = (t & 1) * 128 + hf * HC;
+            float s[HC];
             {
-                uint32_t raw[BLK];
-                if constexpr (BLK == 128) {
-                    tmem_ld128_wait(tmem + lane_base + (t & 1) * 128, raw);
-                } else {
+                uint32_t raw[HC];
+                if constexpr (HC == 64) tmem_ld64_wait(tmem + lane_base + s_col, raw);
+                else tmem_ld32_wait(tmem + lane_base + s_col, raw);
 #pragma unroll
-                    for (int c = 0; c < BLK / 32; ++c) tmem_ld32_wait(tmem + lane_base + (t & 1) * 128 + c * 32, raw + c * 32);
-                }
-#pragma unroll
-                for (int c = 0; c < BLK; ++c) s[c] = __uint_as_float(raw[c]);
+                for (int c = 0; c < HC; ++c) s[c] = __uint_as_float(raw[c]);
             }
-            if (valid < BLK) {                      // ragged last key block only
+            if (valid < HC) {                       // ragged last key block only
 #pragma unroll
-                for (int c = 0; c < BLK; ++c)
+                for (int c = 0; c < HC; ++c)
                     if (c >= valid) s[c] = -INFINITY;
             }
-            // row max: four independent three-input chains over s[4 .. BLK-5], then the
+            // row max: four independent three-input chains over s[4 .. HC-5], then the
             // last four columns
             float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
 #pragma unroll
-            for (int c = 4; c + 8 <= BLK; c += 8) {
+            for (int c = 4; c + 8 <= HC; c += 8) {
                 mx0 = fmax3(mx0, s[c], s[c + 4]);
                 mx1 = fmax3(mx1, s[c + 1], s[c + 5]);
                 mx2 = fmax3(mx2, s[c + 2], s[c + 6]);
                 mx3 = fmax3(mx3, s[c + 3], s[c + 7]);
             }
-            mx0 = fmaxf(mx0, s[BLK - 4]);
-            mx1 = fmaxf(mx1, s[BLK - 3]);
-            mx2 = fmaxf(mx2, s[BLK - 2]);
-            mx3 = fmaxf(mx3, s[BLK - 1]);
+            mx0 = fmaxf(mx0, s[HC - 4]);
+            mx1 = fmaxf(mx1, s[HC - 3]);
+            mx2 = fmaxf(mx2, s[HC - 2]);
+            mx3 = fmaxf(mx3, s[HC - 1]);
             const float mt2 = fmax3(mx0, mx1, fmaxf(mx2, mx3)) * sc;
             const bool upd = mt2 > m_run + kRescaleLog2;
             const float m_new = upd ? mt2 : m_run;
             const float alpha = upd ? ex2_approx(m_run - m_new) : 1.f;
-            // P = 2^(s*scale_log2 - m): packed FMA, MUFU exp2, bf16 pack
-            uint32_t pk[BLK / 2];
-            float ls0 = 0.f, ls1 = 0.f, ls2 = 0.f, ls3 = 0.f;
+            // a half that has seen only masked columns so far keeps m = -inf; its P is 0
+            const float m_sub = m_new == -INFINITY ? 0.f : m_new;
+            // P = 2^(s*scale_log2 - m): packed FMA, MUFU exp2, bf16 pack; the row sum
+            // adds the rounded values (unpacked from the bf16 pair)
+            uint32_t pk[HC / 2];
+            float lr0 = 0.f, lr1 = 0.f, lr2 = 0.f, lr3 = 0.f;
+            float le0 = 0.f, le1 = 0.f;
 #pragma unroll
-            for (int c = 0; c < BLK; c += 2) {
+            for (int c = 0; c < HC; c += 2) {
                 float x0, x1;
-                ffma2(x0, x1, s[c], s[c + 1], sc, sc, -m_new, -m_new);
+                ffma2(x0, x1, s[c], s[c + 1], sc, sc, -m_sub, -m_sub);
                 const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
-                pk[c / 2] = pack_bf16x2(p0, p1);
-                if constexpr (WITH_LSE) {
-                    if ((c & 2) == 0) fadd2(ls0, ls1, ls0, ls1, p0, p1);
-                    else fadd2(ls2, ls3, ls2, ls3, p0, p1);
-                }
+                const uint32_t w = pack_bf16x2(p0, p1);
+                pk[c / 2] = w;
+                const float r0 = __uint_as_float(w << 16), r1 = __uint_as_float(w & 0xFFFF0000u);
+                if ((c & 2) == 0) fadd2(lr0, lr1, lr0, lr1, r0, r1);
+                else fadd2(lr2, lr3, lr2, lr3, r0, r1);
+                if constexpr (WITH_LSE) fadd2(le0, le1, le0, le1, p0, p1);
             }
-            if constexpr (WITH_LSE) l_run = l_run * alpha + ((ls0 + ls1) + (ls2 + ls3));
+            l_run = l_run * alpha + ((lr0 + lr1) + (lr2 + lr3));
+            if constexpr (WITH_LSE) l_ex = l_ex * alpha + (le0 + le1);
             m_run = m_new;
-#pragma unroll
-            for (int c = 0; c < BLK / 32; ++c) tmem_st16(tmem + lane_base + (t & 1) * 128 + c * 16, pk + c * 16);
-            // Consume the completion of PV_{t-1} on every tile.  An mbarrier parity wait is
-            // only unambiguous while the waiter is at most one phase behind; waiting on
-            // every phase keeps it so (PV_t cannot start before this tile's P is ready), and
-            // by now PV_{t-1}, issued before this tile's softmax began, has normally finished.
+            if constexpr (HC == 64) tmem_st32(tmem + lane_base + s_col, *reinterpret_cast<const uint32_t(*)[32]>(pk));
+            else tmem_st16(tmem + lane_base + s_col, pk);
+            // Consume the completion of PV_{t-1} (both halves) on every tile.  An mbarrier
+            // parity wait is only unambiguous while the waiter is at most one phase behind;
+            // waiting on every phase keeps it so (PV_t cannot start before this P is ready),
+            // and by now PV_{t-1} has normally finished.
             if (t > 0) {
                 ok = mbar_wait_warp(bar(L::B_O), (t - 1) & 1, ctl);
                 if (!ok) break;
             }
             if (__any_sync(0xffffffffu, upd && t > 0)) {
-                // rescale [O | rowsum], accumulated through PV_{t-1}, in place
+                // rescale O_h, accumulated through PV_{t-1}, in place
                 tc_fence_after();
                 const float a_row = (upd && t > 0) ? alpha : 1.f;
                 uint32_t raw[32];
 #pragma unroll
-                for (int c = 0; c < (NPV + 31) / 32; ++c) {
-                    tmem_ld32_wait(tmem + lane_base + kTmemO + c * 32, raw);
+                for (int c = 0; c < D / 32; ++c) {
+                    tmem_ld32_wait(tmem + lane_base + o_col + c * 32, raw);
 #pragma unroll
                     for (int e = 0; e < 32; ++e) raw[e] = __float_as_uint(__uint_as_float(raw[e]) * a_row);
-                    tmem_st32(tmem + lane_base + kTmemO + c * 32, raw);
+                    tmem_st32(tmem + lane_base + o_col + c * 32, raw);
                 }
             }
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(bar(L::B_PF + (t & 1)));
         }
-        // ---- epilogue ----
+        // completion of the last PV (the loop consumed every earlier one)
+        if (ok && nkept > 0) ok = mbar_wait_warp(bar(L::B_O), (nkept - 1) & 1, ctl);
+        // ---- merge the two halves and write the output ----
+        float4* xch = reinterpret_cast<float4*>(smem + L::OFF_XCH);
+        xch[hf * kTileM + r] = make_float4(m_run, l_run, l_ex, 0.f);
+        tc_fence_before();
+        named_bar_sync(kBarSoftmax, kSoftmaxThreads);    // every softmax warp gets here
+        tc_fence_after();
         if (__all_sync(0xffffffffu, ok && !*abort_flag)) {
-            const bool row_ok = r < BLK && (i * BLK + r) < Nq;
-            // completion of the last PV (the loop consumed every earlier one)
-            if (nkept > 0) ok = mbar_wait_warp(bar(L::B_O), (nkept - 1) & 1, ctl);
-            if (ok) {
-                tc_fence_after();
-                float lsum = 0.f;
-                if (nkept > 0) {
-                    uint32_t raw[32];
-                    tmem_ld32_wait(tmem + lane_base + kTmemO + D, raw);
-                    lsum = __uint_as_float(raw[0]);
-                }
-                const float inv_l = nkept > 0 ? 1.f / lsum : 0.f;
-                float lse_val = -INFINITY;
-                if constexpr (WITH_LSE) {
-                    if (nkept > 0) lse_val = (m_run + lg2_approx(l_run)) * 0.69314718055994530942f;
-                }
-                // destination rows: the row itself, or every token an anchor stands for
-                int tok0 = 0, ncopy = 0, copy_stride = 0;
-                if (row_ok) {
-                    const int a = i * BLK + r;
-                    if (!rep) {
-                        tok0 = a;
-                        ncopy = 1;
-                    } else {
-                        const int nva = p.F * p.Ar * p.Wl;
-                        tok0 = anchor_token(p, a);
-                        if (a < nva) {
-                            const int ya = (a / p.Wl) % p.Ar;
-                            ncopy = min(p.stride, p.Hl - ya * p.stride);
-                            copy_stride = p.Wl;
-                        } else {
-                            ncopy = 1;
-                        }
-                    }
-                }
-#pragma unroll
-                for (int c = 0; c < D / 32; ++c) {
-                    uint32_t raw[32];
-                    if (nkept > 0) {
-                        tmem_ld32_wait(tmem + lane_base + kTmemO + c * 32, raw);
-                    } else {
-#pragma unroll
-                        for (int e = 0; e < 32; ++e) raw[e] = 0u;
-                    }
-                    if (p.out_f32) {
-#pragma unroll
-                        for (int e = 0; e < 32; ++e) raw[e] = __float_as_uint(__uint_as_float(raw[e]) * inv_l);
-                        for (int cp = 0; cp < ncopy; ++cp) {
-                            const size_t tok = static_cast<size_t>(tok0 + cp * copy_stride);
-                            store_row32_f32(reinterpret_cast<float*>(p.o) + (static_cast<size_t>(h) * p.N + tok) * D +
-                                                c * 32, raw);
-                        }
-                    } else {
-                        uint32_t packed[16];
-#pragma unroll
-                        for (int e = 0; e < 16; ++e)
-                            packed[e] = pack_bf16x2(__uint_as_float(raw[2 * e]) * inv_l,
-                                                    __uint_as_float(raw[2 * e + 1]) * inv_l);
-                        for (int cp = 0; cp < ncopy; ++cp) {
-                            const size_t tok = static_cast<size_t>(tok0 + cp * copy_stride);
-                            store_row32_bf16(p.o + (static_cast<size_t>(h) * p.N + tok) * D + c * 32, packed);
-                        }
-                    }
-                }
-                if (p.lse)
-                    for (int cp = 0; cp < ncopy; ++cp)
-                        p.lse[static_cast<size_t>(h) * p.N + tok0 + cp * copy_stride] = lse_val;
+            const float4 x0 = xch[r], x1 = xch[kTileM + r];
+            const float m = fmaxf(x0.x, x1.x);
+            const float w0 = x0.x == -INFINITY ? 0.f : ex2_approx(x0.x - m);
+            const float w1 = x1.x == -INFINITY ? 0.f : ex2_approx(x1.x - m);
+            const float lsum = x0.y * w0 + x1.y * w1;
+            const float inv_l = nkept > 0 ? 1.f / lsum : 0.f;
+            const float c0 = w0 * inv_l, c1 = w1 * inv_l;
+            float lse_val = -INFINITY;
+            if constexpr (WITH_LSE) {
+                if (nkept > 0) lse_val = (m + lg2_approx(x0.z * w0 + x1.z * w1)) * 0.69314718055994530942f;
             }
+            const bool row_ok = r < BLK && (i * BLK + r) < Nq;
+            // destination rows: the row itself, or every token an anchor stands for
+            int tok0 = 0, ncopy = 0, copy_stride = 0;
+            if (row_ok) {
+                const int a = i * BLK + r;
+                if (!rep) {
+                    tok0 = a;
+                    ncopy = 1;
+                } else {
+                    const int nva = p.F * p.Ar * p.Wl;
+                    tok0 = anchor_token(p, a);
+                    if (a < nva) {
+                        const int ya = (a / p.Wl) % p.Ar;
+                        ncopy = min(p.stride, p.Hl - ya * p.stride);
+                        copy_stride = p.Wl;
+                    } else {
+                        ncopy = 1;
+                    }
+                }
+            }
+            // this warp writes output columns [hf*D/2, (hf+1)*D/2), reading both halves
+#pragma unroll
+            for (int cc = 0; cc < D / 64; ++cc) {
+                const int c = hf * (D / 64) + cc;             // 32-column chunk index
+                uint32_t raw[32];
+                if (nkept > 0) {
+                    uint32_t raw1[32];
+                    tmem_ld32_wait(tmem + lane_base + kTmemO + c * 32, raw);
+                    tmem_ld32_wait(tmem + lane_base + kTmemO + D + c * 32, raw1);
+#pragma unroll
+                    for (int e = 0; e < 32; e += 2) {
+                        float y0, y1, z0, z1;
+                        ffma2(y0, y1, __uint_as_float(raw1[e]), __uint_as_float(raw1[e + 1]), c1, c1, 0.f, 0.f);
+                        ffma2(z0, z1, __uint_as_float(raw[e]), __uint_as_float(raw[e + 1]), c0, c0, y0, y1);
+                        raw[e] = __float_as_uint(z0);
+                        raw[e + 1] = __float_as_uint(z1);
+                    }
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) raw[e] = 0u;
+                }
+                if (p.out_f32) {
+                    for (int cp = 0; cp < ncopy; ++cp) {
+                        const size_t tok = static_cast<size_t>(tok0 + cp * copy_stride);
+                        store_row32_f32(reinterpret_cast<float*>(p.o) + (static_cast<size_t>(h) * p.N + tok) * D +
+                                            c * 32, raw);
+                    }
+                } else {
+                    uint32_t packed[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e)
+                        packed[e] = pack_bf16x2(__uint_as_float(raw[2 * e]), __uint_as_float(raw[2 * e + 1]));
+                    for (int cp = 0; cp < ncopy; ++cp) {
+                        const size_t tok = static_cast<size_t>(tok0 + cp * copy_stride);
+                        store_row32_bf16(p.o + (static_cast<size_t>(h) * p.N + tok) * D + c * 32, packed);
+                    }
+                }
+            }
+            if (p.lse && hf == 0)
+                for (int cp = 0; cp < ncopy; ++cp)
+                    p.lse[static_cast<size_t>(h) * p.N + tok0 + cp * copy_stride] = lse_val;
         }
     }
 

@@ -118,6 +118,15 @@ __device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, co
     return __all_sync(0xffffffffu, ok);
 }
 
+// Second half of a split wait: `tok` is each lane's mbar_try_wait result for the same
+// phase, issued earlier so that its latency overlapped other work.  The phase being waited
+// for must be the barrier's current or next one (never two phases ahead of the last one
+// this warp consumed), or the parity test would be ambiguous.
+__device__ __forceinline__ bool mbar_wait_warp_tok(uint32_t bar, uint32_t parity, bool tok, const WaitCtl& ctl) {
+    if (__all_sync(0xffffffffu, tok)) return true;
+    return mbar_wait_warp(bar, parity, ctl);
+}
+
 // Wait used only while draining after an abort: bounded by its own limit, never sets
 // the abort flag (it is already set).
 __device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
