@@ -39,7 +39,11 @@ UNIT = "TFLOPS"
 # DRAM bytes (read + write) of one attn_fwd_kernel launch on the wan13b workload, from an
 # ncu capture (profiles/attn_fwd_wan13b.md), valid only for the kernel sources it was taken
 # on: reported as roofline.traffic while the source hashes still match, else null.
-NCU_TRAFFIC = {("wan13b", "70b321627e5a", "e4390e39220d"): 302_647_040 + 86_838_016}
+NCU_TRAFFIC = {("wan13b", "3416fe395751", "a9ea2ee30fca"): 302_676_480 + 86_866_176}
+
+# MUFU exp2 throughput of one SM: 4 lanes per clock in each of the 4 sub-partitions.
+MUFU_EX2_PER_CLK_SM = 16
+B200_SMS = 148
 
 
 def _src_sha(name):
@@ -186,6 +190,20 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def run_energy_only(args, wl, dev, torch, ops, synth):
+    """The calibration leg alone: fused row-LSE + block-energy pass (two passes over K)."""
+    s = wl.shape
+    H = args.heads or s.H
+    q, k, _ = synth.make_qkv(wl, device=dev, heads=H)
+    E = ops.block_energy(q, k, s.block)
+    ms = _time_calls(lambda: ops.block_energy(q, k, s.block, out=E), args.steps, args.warmup, torch)
+    ops.device_check()
+    exps = 2.0 * s.N * s.N * H / (ms * 1e-3)
+    peak = MUFU_EX2_PER_CLK_SM * B200_SMS * 1965.0e6
+    print(json.dumps({"leg": "block_energy", "workload": wl.name, "H": H, "N": s.N, "D": s.D, "block": s.block,
+                      "ms": ms, "exp2_per_s": exps, "frac_of_mufu_at_1965mhz": exps / peak}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -196,6 +214,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true", help="skip dense / e2e / calibration legs")
+    ap.add_argument("--energy-only", action="store_true",
+                    help="time only the fused LSE + block-energy pass (calibration) and print its own line")
+    ap.add_argument("--heads", type=int, default=None, help="with --energy-only: the first H heads only")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -219,6 +240,8 @@ def main():
     wl = synth.WORKLOADS[args.workload]
     s = wl.shape
     B, D, N, H = s.block, s.D, s.N, s.H
+    if args.energy_only:
+        return run_energy_only(args, wl, dev, torch, ops, synth)
     q, k, v = synth.make_qkv(wl, device=dev)
     mask_np = synth.make_head_masks(wl, timestep=args.timestep)
     mask = torch.from_numpy(mask_np).to(dev)
@@ -320,10 +343,16 @@ def main():
             msk = torch.empty(energy.shape, dtype=torch.uint8, device=dev)
             ms_sel = _time_calls(lambda: ops.select_mask(energy, 0.95, out=msk), 20, 3, torch)
             sel_bytes = energy.numel() * 4 + msk.numel()
+            exps = 2.0 * N * N * H / (ms_energy * 1e-3)
+            clk_mhz = (clk.summary().get("sm_max_mhz") or 1965.0)
+            mufu_peak = MUFU_EX2_PER_CLK_SM * B200_SMS * clk_mhz * 1e6
             extras["calibration"] = {
                 "energy_ms": ms_energy,
                 "energy_tflops_qk": 2 * 2.0 * N * N * D * H / (ms_energy * 1e-3) / 1e12,
-                "energy_exps_per_s": 2.0 * N * N * H / (ms_energy * 1e-3),
+                "energy_exps_per_s": exps,
+                "energy_roofline": {"bound": "alu", "unit": "exp2/s", "achieved": exps, "peak": mufu_peak,
+                                    "frac": exps / mufu_peak, "kernel": f"block_energy_kernel<{D},{B},4>",
+                                    "peak_source": "16 MUFU ex2 per clock per SM x 148 SMs x max SM clock"},
                 "select_ms": ms_sel, "select_gbs": sel_bytes / (ms_sel * 1e-3) / 1e9,
                 "select_frac_hbm": sel_bytes / (ms_sel * 1e-3) / 1e9 / peaks["hbm_gbs"],
                 "tau": 0.95, "selected_density": float(msk.float().mean().item())}
@@ -342,7 +371,7 @@ def main():
                      "unit": "TFLOP/s", "frac": value / world / peaks["bf16_tflops"],
                      "traffic": NCU_TRAFFIC.get((wl.name, _src_sha("attn_fwd.cuh"), _src_sha("ptx.cuh"))),
                      "algorithmic_bytes": 4 * q.numel() * q.element_size(),
-                     "peak_source": f"{peaks['source']} bf16 burst", "kernel": f"attn_fwd_kernel<{D},{B},2,2,0>",
+                     "peak_source": f"{peaks['source']} bf16 burst", "kernel": f"attn_fwd_kernel<{D},{B},3,3,0>",
                      "frac_of_sustained": value / world / peaks["bf16_tflops_sustained"]},
         "gpu_launches": args.steps,
         "clocks": clk.summary(),

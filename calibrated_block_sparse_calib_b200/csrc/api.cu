@@ -98,11 +98,7 @@ calib_status launch_status() {
 template <int D, int BLK, bool WITH_LSE>
 calib_status launch_attn(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                          const calib::AttnParams& p, int grid, cudaStream_t st) {
-#ifndef CALIB_ATTN_KST
-#define CALIB_ATTN_KST 3
-#define CALIB_ATTN_VST 3
-#endif
-    constexpr int KST = CALIB_ATTN_KST, VST = CALIB_ATTN_VST;
+    constexpr int KST = 3, VST = 3;   // K / V ring depths
     using L = calib::AttnSmem<D, BLK, KST, VST>;
     static_assert(L::BYTES <= 232448, "shared memory budget");
     auto* fn = calib::attn_fwd_kernel<D, BLK, KST, VST, WITH_LSE>;
@@ -167,13 +163,13 @@ calib_status attn_common(const void* q, const void* k, const void* v, void* o, f
 
 // ---- energy ------------------------------------------------------------------------
 template <int D, int BLK>
-calib_status launch_energy(const CUtensorMap& tq, const CUtensorMap& tk, const calib::EnergyParams& p,
-                           int grid, cudaStream_t st) {
-    constexpr int KST = 3;
+calib_status launch_energy(const CUtensorMap& tk, const calib::EnergyParams& p, int grid, cudaStream_t st) {
+    constexpr int KST = 4;
     using L = calib::EnergySmem<D, BLK, KST>;
+    static_assert(L::BYTES <= 232448, "shared memory budget");
     auto* fn = calib::block_energy_kernel<D, BLK, KST>;
     if (calib_status s = ensure_smem(reinterpret_cast<const void*>(fn), L::BYTES)) return s;
-    fn<<<grid, calib::kEnergyThreads, L::BYTES, st>>>(tq, tk, p);
+    fn<<<grid, calib::kEnergyThreads, L::BYTES, st>>>(tk, p);
     return launch_status();
 }
 
@@ -218,6 +214,7 @@ calib_status calib_block_energy(const void* q, const void* k, const float* lse, 
     if (q_rows && n_q < 1) return CALIB_ERR_INVALID;
     const int nq = cdiv(Nq, block), nk = cdiv(N, block);
     if (static_cast<long long>(H) * nq > (1ll << 31) - 1) return CALIB_ERR_INVALID;
+    if (N > calib::kEnergyMaxTokens) return CALIB_ERR_UNSUPPORTED;
     if (calib_status s = check_device()) return s;
     calib::EnergyParams p{};
     p.q = static_cast<const __nv_bfloat16*>(q);
@@ -228,13 +225,12 @@ calib_status calib_block_energy(const void* q, const void* k, const float* lse, 
     p.accumulate = accumulate ? 1 : 0;
     p.scale_log2 = scale * 1.4426950408889634f;
     p.timeout_ns = kDefaultTimeoutNs;
-    CUtensorMap tq, tk;
-    if (!make_tmap(&tq, q, D, N, H, calib::kTileM) || !make_tmap(&tk, k, D, N, H, block)) return CALIB_ERR_CUDA;
+    CUtensorMap tk;
+    if (!make_tmap(&tk, k, D, N, H, block)) return CALIB_ERR_CUDA;
     cudaStream_t st = as_stream(stream);
     const int grid = H * nq;
-    if (D == 128) return block == 128 ? launch_energy<128, 128>(tq, tk, p, grid, st)
-                                      : launch_energy<128, 64>(tq, tk, p, grid, st);
-    return block == 128 ? launch_energy<64, 128>(tq, tk, p, grid, st) : launch_energy<64, 64>(tq, tk, p, grid, st);
+    if (D == 128) return block == 128 ? launch_energy<128, 128>(tk, p, grid, st) : launch_energy<128, 64>(tk, p, grid, st);
+    return block == 128 ? launch_energy<64, 128>(tk, p, grid, st) : launch_energy<64, 64>(tk, p, grid, st);
 }
 
 calib_status calib_select_mask(const float* energy, int H, int nq, int nk, double tau, const uint8_t* force_keep,

@@ -6,15 +6,25 @@
 // stored:  E[h,i,j] = sum_{r in I_i} sum_{c in J_j} 2^(x_rc - lse2_r),  x = s * scale*log2(e),
 // lse2 = LSE / ln 2.
 //
-// One CTA per (head h, query block i), 192 threads:
-//   warp 0      TMA: Q tile (unless the rows are gathered), then K_j for every key block,
-//               twice when the LSE is not supplied (pass 1 computes it, pass 2 sums).
-//   warp 1      TMEM owner (256 columns: two S buffers) and MMA issuer, S = Q K_j^T.
-//   warps 2..5  one row per thread: pass 1 keeps an exact running max / sum and ends with
-//               the row's LSE in a register (the LSE is never written to memory, so no
-//               scratch buffer is needed); pass 2 sums 2^(x - lse2) over the tile's valid
-//               columns, reduces the 128 rows (warp shuffles, then 4 partials in fixed
-//               order) and writes one energy per tile.
+// One CTA per (head h, query block i), 320 threads:
+//   warp 0      TMA: K_j for every key block, twice when the LSE is not supplied (pass 1
+//               computes it, pass 2 sums the blocks).
+//   warp 1      TMEM owner (512 columns) and MMA issuer (one elected lane of the converged
+//               warp): S = Q K_j^T as a TS MMA, M=128, N=B, K=D.  Q sits in tensor memory
+//               as packed bf16 pairs, so only K is read from shared memory (an SS MMA also
+//               re-reads Q from shared memory for every key block, and at M=N=128 the
+//               operand reads, not the math, set its rate).  S rotates through three
+//               buffers; a buffer is handed back as soon as its tile is in registers.
+//   warps 2..9  arithmetic.  A query row (TMEM lane) is split between two warps, each
+//               owning half of every tile's columns.  Pass 1: each half keeps an exact
+//               running (max, sum) of 2^x over its columns; the halves are merged once, at
+//               the end of the pass, into the row's LSE (kept in a register: the LSE is
+//               never written to memory, so no scratch buffer is needed).  Pass 2: each
+//               thread sums 2^(x - lse2) over its columns; each warp reduces its 32 rows
+//               with shuffles, batched over four key blocks, into a shared-memory table of
+//               per-warp partials, and after the last key block the CTA adds the eight
+//               partials of every block in a fixed order and writes the row of energies.
+// Tensor memory: S buffers at columns [0,128), [128,256), [256,384); Q at [384, 384+D/2).
 // [AdaSpa] §2 caches the LSE to reuse it in a later search; a supplied LSE skips pass 1.
 #pragma once
 #include <cuda_bf16.h>
@@ -23,11 +33,18 @@
 
 namespace calib {
 
-constexpr uint32_t kEnergyTmemCols = 256;
-constexpr int kEnergyThreads = 192;
+constexpr int kEnergyGroups = 2;                          // column halves per row
+constexpr int kEnergySoftmaxWarps = 4 * kEnergyGroups;    // 8
+constexpr int kEnergySoftmaxThreads = 32 * kEnergySoftmaxWarps;
+constexpr int kEnergyThreads = 64 + kEnergySoftmaxThreads;
+constexpr int kEnergySBufs = 3;
+constexpr uint32_t kEnergyTmemCols = 512;
+constexpr uint32_t kEnergyTmemQ = 384;
+constexpr int kEnergyMaxTokens = 131072;                 // N limit (per-block partial table)
+constexpr uint32_t kBarEnergy = 1;                        // named barrier of the arithmetic warps
 
 struct EnergyParams {
-    const __nv_bfloat16* q;   // [H, N, D] (read directly only for gathered rows)
+    const __nv_bfloat16* q;   // [H, N, D]
     const int32_t* q_rows;    // [n_q] token indices or nullptr
     const float* lse_in;      // [H, Nq] natural-log LSE or nullptr
     float* energy;            // [H, nq, nk]
@@ -40,55 +57,55 @@ struct EnergyParams {
 template <int D, int BLK, int KST>
 struct EnergySmem {
     static constexpr int CH = D / 64;
-    static constexpr uint32_t Q_BYTES = CH * kTileM * 128;
     static constexpr uint32_t K_BYTES = CH * BLK * 128;
-    static constexpr uint32_t OFF_K = Q_BYTES;
-    static constexpr uint32_t OFF_BAR = OFF_K + KST * K_BYTES;
-    static constexpr int B_Q = 0, B_KF = 1, B_KE = B_KF + KST, B_SF = B_KE + KST, B_SE = B_SF + 2,
-                         B_DRAIN = B_SE + 2, NBARS = B_DRAIN + 1;
-    static constexpr uint32_t OFF_RED = OFF_BAR + NBARS * 8;      // float red[2][4]
-    static constexpr uint32_t OFF_MISC = OFF_RED + 32;
-    // at least 80 KB: two CTAs of 256 TMEM columns each per SM
-    static constexpr uint32_t RAW = OFF_MISC + 16 + 1024;
-    static constexpr uint32_t BYTES = RAW > 80u * 1024 ? RAW : 80u * 1024;
+    static constexpr uint32_t OFF_K = 0;
+    static constexpr int MAX_NK = kEnergyMaxTokens / BLK;
+    static constexpr uint32_t OFF_RED = KST * K_BYTES;    // float [warps][MAX_NK]
+    static constexpr uint32_t OFF_XCH = OFF_RED + kEnergySoftmaxWarps * MAX_NK * 4;   // float2 [groups][128]
+    static constexpr uint32_t OFF_BAR = OFF_XCH + kEnergyGroups * kTileM * 8;
+    static constexpr int B_Q = 0, B_KF = 1, B_KE = B_KF + KST, B_SF = B_KE + KST, B_SE = B_SF + kEnergySBufs,
+                         B_DRAIN = B_SE + kEnergySBufs, NBARS = B_DRAIN + 1;
+    static constexpr uint32_t OFF_MISC = OFF_BAR + NBARS * 8;   // tmem base, abort flag
+    static constexpr uint32_t BYTES = OFF_MISC + 16 + 1024;    // + alignment slack
 };
 
 template <int D, int BLK, int KST>
 __global__ void __launch_bounds__(kEnergyThreads, 1)
-block_energy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                    const EnergyParams p) {
+block_energy_kernel(const __grid_constant__ CUtensorMap tm_k, const EnergyParams p) {
     using L = EnergySmem<D, BLK, KST>;
     constexpr int CH = L::CH;
+    constexpr int HC = BLK / kEnergyGroups;               // columns per thread and tile
+    constexpr int SB = kEnergySBufs;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
-    uint8_t* sQ = smem;
     uint8_t* sK = smem + L::OFF_K;
+    float* red = reinterpret_cast<float*>(smem + L::OFF_RED);
+    float2* xch = reinterpret_cast<float2*>(smem + L::OFF_XCH);
     const uint32_t bar0 = smem_u32(smem + L::OFF_BAR);
     auto bar = [&](int idx) -> uint32_t { return bar0 + 8u * idx; };
-    float* red = reinterpret_cast<float*>(smem + L::OFF_RED);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
 
     const uint32_t warp = warp_id(), lane = lane_id();
     const int h = blockIdx.x / p.nq;
     const int i = blockIdx.x - h * p.nq;
-    const bool gather = p.q_rows != nullptr;
     const bool two_pass = p.lse_in == nullptr;
-    const int n_iter = p.nk * (two_pass ? 2 : 1);
+    const int nk = p.nk;
+    const int n_iter = nk * (two_pass ? 2 : 1);
 
     if (threadIdx.x == 0) {
-        mbar_init(bar(L::B_Q), gather ? 128u : 1u);
+        mbar_init(bar(L::B_Q), 128);
         for (int s = 0; s < KST; ++s) { mbar_init(bar(L::B_KF + s), 1); mbar_init(bar(L::B_KE + s), 1); }
-        for (int b = 0; b < 2; ++b) { mbar_init(bar(L::B_SF + b), 1); mbar_init(bar(L::B_SE + b), 128); }
+        for (int b = 0; b < SB; ++b) {
+            mbar_init(bar(L::B_SF + b), 1);
+            mbar_init(bar(L::B_SE + b), kEnergySoftmaxThreads);
+        }
         mbar_init(bar(L::B_DRAIN), 1);
         *abort_flag = 0;
         fence_barrier_init();
     }
-    if (warp == 0 && lane == 0) {
-        tma_prefetch_desc(&tm_q);
-        tma_prefetch_desc(&tm_k);
-    }
+    if (warp == 0 && lane == 0) tma_prefetch_desc(&tm_k);
     if (warp == 1) {
         tmem_alloc(smem_u32(tmem_slot), kEnergyTmemCols);
         tmem_relinquish();
@@ -99,131 +116,203 @@ block_energy_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     const uint32_t tmem = *tmem_slot;
     const WaitCtl ctl{abort_flag, p.timeout_ns};
 
-    int armed_q = 0, armed_k[KST];
+    int armed_k[KST];
 #pragma unroll
     for (int s = 0; s < KST; ++s) armed_k[s] = 0;
 
     if (warp == 0) {
-        if (lane == 0) {
-            if (!gather) {
-                mbar_arrive_expect_tx(bar(L::B_Q), L::Q_BYTES);
-                for (int c = 0; c < CH; ++c)
-                    tma_load_3d(smem_u32(sQ + c * kTileM * 128), &tm_q, bar(L::B_Q), c * 64, i * BLK, h);
-                armed_q = 1;
-            }
-            for (int t = 0; t < n_iter; ++t) {
-                const int s = t % KST;
-                if (!mbar_wait(bar(L::B_KE + s), ((t / KST) & 1) ^ 1, ctl)) break;
-                const int j = t % p.nk;
+        // ===================== TMA producer (converged warp, one elected lane issues) ====
+        for (int t = 0; t < n_iter; ++t) {
+            const int s = t % KST;
+            if (!mbar_wait_warp(bar(L::B_KE + s), ((t / KST) & 1) ^ 1, ctl)) break;
+            const int j = t < nk ? t : t - nk;
+            if (elect_one()) {
                 mbar_arrive_expect_tx(bar(L::B_KF + s), L::K_BYTES);
                 for (int c = 0; c < CH; ++c)
-                    tma_load_3d(smem_u32(sK + s * L::K_BYTES + c * BLK * 128), &tm_k, bar(L::B_KF + s),
-                                c * 64, j * BLK, h);
-                ++armed_k[s];
+                    tma_load_3d(smem_u32(sK + s * L::K_BYTES + c * BLK * 128), &tm_k, bar(L::B_KF + s), c * 64,
+                                j * BLK, h);
             }
+            ++armed_k[s];
         }
     } else if (warp == 1) {
-        if (lane == 0) {
-            constexpr uint32_t idesc_qk = idesc_bf16_f32(kTileM, BLK, false, false);
-            const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK);
-            bool ok = mbar_wait(bar(L::B_Q), 0, ctl);
-            for (int t = 0; ok && t < n_iter; ++t) {
-                const int s = t % KST, b = t & 1, u = t >> 1;
-                if (u >= 1 && !(ok = mbar_wait(bar(L::B_SE + b), (u - 1) & 1, ctl))) break;
-                if (!(ok = mbar_wait(bar(L::B_KF + s), (t / KST) & 1, ctl))) break;
-                tc_fence_after();
+        // ===================== MMA issuer ===============================================
+        constexpr uint32_t idesc_qk = idesc_bf16_f32(kTileM, BLK, false, false);
+        const uint32_t sKa = smem_u32(sK);
+        bool ok = mbar_wait_warp(bar(L::B_Q), 0, ctl);
+        for (int t = 0; ok && t < n_iter; ++t) {
+            const int s = t % KST, b = t % SB, u = t / SB;
+            ok = mbar_wait_warp(bar(L::B_KF + s), (t / KST) & 1, ctl);
+            // S buffer b is free once every arithmetic thread has loaded its previous tile
+            if (ok && u >= 1) ok = mbar_wait_warp(bar(L::B_SE + b), (u - 1) & 1, ctl);
+            if (!ok) break;
+            tc_fence_after();
+            if (elect_one()) {
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t inner = (kk & 3) * 32;
-                    const uint64_t ad = smem_desc_sw128(sQa + (kk >> 2) * kTileM * 128 + inner, 16, 1024);
                     const uint64_t bd =
-                        smem_desc_sw128(sKa + s * L::K_BYTES + (kk >> 2) * BLK * 128 + inner, 16, 1024);
-                    umma_ss(tmem + b * 128, ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
+                        smem_desc_sw128(sKa + s * L::K_BYTES + (kk >> 2) * BLK * 128 + (kk & 3) * 32, 16, 1024);
+                    umma_ts(tmem + b * 128, tmem + kEnergyTmemQ + kk * 8, bd, idesc_qk, kk > 0 ? 1u : 0u);
                 }
                 umma_commit(bar(L::B_SF + b));
                 umma_commit(bar(L::B_KE + s));
             }
         }
     } else {
+        // ===================== arithmetic (warps 2..9) ==================================
+        const int g = static_cast<int>(warp - 2) >> 2;      // column half of every tile
+        const int widx = static_cast<int>(warp) - 2;        // partial-sum table row
         const uint32_t q4 = warp & 3;
-        const int r = static_cast<int>(q4 * 32 + lane);
+        const int r = static_cast<int>(q4 * 32 + lane);     // tile row == TMEM lane
         const uint32_t lane_base = (q4 * 32) << 16;
-        const int qrow = i * BLK + r;                      // row in the query sequence
+        const int qrow = i * BLK + r;                       // row in the query sequence
         const bool row_ok = r < BLK && qrow < p.Nq;
-        if (gather) {
-            const __nv_bfloat16* src =
-                (qrow < p.Nq) ? p.q + (static_cast<size_t>(h) * p.N + p.q_rows[qrow]) * D : nullptr;
-            gather_q_row<D>(sQ, r, src);
-            fence_proxy_async_smem();
+        const float sc = p.scale_log2;
+        if (g == 0) {
+            // Q row -> tensor memory: bf16 pairs in memory order are the packed TS operand
+            uint32_t w[32];
+            const uint4* src = row_ok ? reinterpret_cast<const uint4*>(
+                                            p.q + (static_cast<size_t>(h) * p.N + (p.q_rows ? p.q_rows[qrow] : qrow)) * D)
+                                      : nullptr;
+#pragma unroll
+            for (int c = 0; c < D / 64; ++c) {
+#pragma unroll
+                for (int v = 0; v < 8; ++v) {
+                    const uint4 x = src ? __ldg(src + c * 8 + v) : make_uint4(0, 0, 0, 0);
+                    w[4 * v] = x.x;
+                    w[4 * v + 1] = x.y;
+                    w[4 * v + 2] = x.z;
+                    w[4 * v + 3] = x.w;
+                }
+                tmem_st32(tmem + lane_base + kEnergyTmemQ + c * 32, w);
+            }
+            tmem_wait_st();
+            tc_fence_before();
             mbar_arrive(bar(L::B_Q));
         }
-        float m_run = -INFINITY, l_run = 0.f, lse2 = 0.f;
-        if (!two_pass && row_ok) lse2 = p.lse_in[static_cast<size_t>(h) * p.Nq + qrow] * 1.4426950408889634f;
-        // After a timeout ("dead") a warp keeps iterating without touching tensor memory,
-        // so the per-tile named barrier below still sees all 128 threads.
-        bool dead = false;
-        for (int t = 0; t < n_iter; ++t) {
-            const int b = t & 1;
-            const int j = t % p.nk;
-            const bool pass_lse = two_pass && t < p.nk;
-            const int valid = min(BLK, p.N - j * BLK);
-            if (!dead) dead = !mbar_wait_warp(bar(L::B_SF + b), (t >> 1) & 1, ctl);
-            float s[BLK];
-            if (!dead) {
-                tc_fence_after();
-                uint32_t raw[32];
+
+        bool ok = true;
+        // Wait for tile t, load this thread's HC columns, hand the S buffer back, mask the
+        // columns past N (ragged last key block only).
+        auto load_tile = [&](int t, int j, float (&s)[HC]) -> bool {
+            const int b = t % SB;
+            if (!mbar_wait_warp(bar(L::B_SF + b), (t / SB) & 1, ctl)) return false;
+            tc_fence_after();
+            {
+                uint32_t raw[HC];
+                if constexpr (HC == 64) tmem_ld64_wait(tmem + lane_base + b * 128 + g * HC, raw);
+                else tmem_ld32_wait(tmem + lane_base + b * 128 + g * HC, raw);
 #pragma unroll
-                for (int c = 0; c < BLK / 32; ++c) {
-                    tmem_ld32_wait(tmem + lane_base + b * 128 + c * 32, raw);
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) s[c * 32 + e] = __uint_as_float(raw[e]);
-                }
-            } else {
-#pragma unroll
-                for (int c = 0; c < BLK; ++c) s[c] = 0.f;
+                for (int c = 0; c < HC; ++c) s[c] = __uint_as_float(raw[c]);
             }
             tc_fence_before();
-            mbar_arrive(bar(L::B_SE + b));          // S buffer may be overwritten now
-            if (pass_lse) {
-                float mt = -INFINITY;
+            mbar_arrive(bar(L::B_SE + b));
+            const int valid = min(BLK, p.N - j * BLK) - g * HC;
+            if (valid < HC) {
 #pragma unroll
-                for (int c = 0; c < BLK; ++c)
-                    if (c < valid) mt = fmaxf(mt, s[c]);
-                const float m_new = fmaxf(m_run, mt * p.scale_log2);
-                float sum = 0.f;
+                for (int c = 0; c < HC; ++c)
+                    if (c >= valid) s[c] = -INFINITY;
+            }
+            return true;
+        };
+        // sum_c 2^(s_c * sc - m) with four independent packed accumulators
+        auto exp_sum = [&](const float (&s)[HC], float m) -> float {
+            float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
 #pragma unroll
-                for (int c = 0; c < BLK; ++c)
-                    if (c < valid) sum += ex2_approx(fmaf(s[c], p.scale_log2, -m_new));
-                l_run = l_run * ex2_approx(m_run - m_new) + sum;
+            for (int c = 0; c < HC; c += 4) {
+                float x0, x1, x2, x3;
+                ffma2(x0, x1, s[c], s[c + 1], sc, sc, -m, -m);
+                ffma2(x2, x3, s[c + 2], s[c + 3], sc, sc, -m, -m);
+                fadd2(a0, a1, a0, a1, ex2_approx(x0), ex2_approx(x1));
+                fadd2(a2, a3, a2, a3, ex2_approx(x2), ex2_approx(x3));
+            }
+            return (a0 + a1) + (a2 + a3);
+        };
+
+        float lse2 = 0.f;
+        if (two_pass) {
+            // ---- pass 1: exact running (max, sum) of this half of the row ----
+            float m_run = -INFINITY, l_run = 0.f;
+            for (int t = 0; t < nk; ++t) {
+                float s[HC];
+                ok = load_tile(t, t, s);
+                if (!ok) break;
+                float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
+#pragma unroll
+                for (int c = 4; c + 8 <= HC; c += 8) {
+                    mx0 = fmax3(mx0, s[c], s[c + 4]);
+                    mx1 = fmax3(mx1, s[c + 1], s[c + 5]);
+                    mx2 = fmax3(mx2, s[c + 2], s[c + 6]);
+                    mx3 = fmax3(mx3, s[c + 3], s[c + 7]);
+                }
+                mx0 = fmaxf(mx0, s[HC - 4]);
+                mx1 = fmaxf(mx1, s[HC - 3]);
+                mx2 = fmaxf(mx2, s[HC - 2]);
+                mx3 = fmaxf(mx3, s[HC - 1]);
+                const float m_new = fmaxf(m_run, fmax3(mx0, mx1, fmaxf(mx2, mx3)) * sc);
+                // a half that has seen only masked columns keeps m = -inf and sum 0
+                const float m_sub = m_new == -INFINITY ? 0.f : m_new;
+                const float alpha = m_run == -INFINITY ? 0.f : ex2_approx(m_run - m_new);
+                l_run = l_run * alpha + exp_sum(s, m_sub);
                 m_run = m_new;
-                if (t == p.nk - 1) lse2 = m_run + lg2_approx(l_run);
-            } else {
-                float e = 0.f;
-                if (row_ok) {
+            }
+            xch[g * kTileM + r] = make_float2(m_run, l_run);
+            named_bar_sync(kBarEnergy, kEnergySoftmaxThreads);
+            float m = -INFINITY;
 #pragma unroll
-                    for (int c = 0; c < BLK; ++c)
-                        if (c < valid) e += ex2_approx(fmaf(s[c], p.scale_log2, -lse2));
-                }
+            for (int gg = 0; gg < kEnergyGroups; ++gg) m = fmaxf(m, xch[gg * kTileM + r].x);
+            float lsum = 0.f;
 #pragma unroll
-                for (int off = 16; off > 0; off >>= 1) e += __shfl_xor_sync(0xffffffffu, e, off);
-                if (lane == 0) red[b * 4 + q4] = e;
-                // red[] is double-buffered: a warp reaches the next write to red[b] only
-                // after the following tile's barrier, which the reader joins after reading.
-                named_bar_sync(1, 128);
-                if (warp == 2 && lane == 0 && !dead) {
-                    const float tot = ((red[b * 4 + 0] + red[b * 4 + 1]) + red[b * 4 + 2]) + red[b * 4 + 3];
-                    float* dst = p.energy + (static_cast<size_t>(h) * p.nq + i) * p.nk + j;
-                    *dst = p.accumulate ? *dst + tot : tot;
+            for (int gg = 0; gg < kEnergyGroups; ++gg) {
+                const float2 v = xch[gg * kTileM + r];
+                if (v.x != -INFINITY) lsum += v.y * ex2_approx(v.x - m);
+            }
+            lse2 = m + lg2_approx(lsum);
+        } else if (row_ok) {
+            lse2 = p.lse_in[static_cast<size_t>(h) * p.Nq + qrow] * 1.4426950408889634f;
+        }
+
+        // ---- pass 2: block sums, reduced per warp in batches of four key blocks ----
+        const int t0 = two_pass ? nk : 0;
+        for (int jb = 0; ok && jb < nk; jb += 4) {
+            float e4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int j = jb + q;
+                if (j < nk && ok) {
+                    float s[HC];
+                    ok = load_tile(t0 + j, j, s);
+                    if (ok && row_ok) e4[q] = exp_sum(s, lse2);
                 }
+            }
+            if (!__all_sync(0xffffffffu, ok)) break;
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) {
+#pragma unroll
+                for (int q = 0; q < 4; ++q) e4[q] += __shfl_xor_sync(0xffffffffu, e4[q], off);
+            }
+            if (lane == 0) {
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    if (jb + q < nk) red[widx * L::MAX_NK + jb + q] = e4[q];
+            }
+        }
+        named_bar_sync(kBarEnergy, kEnergySoftmaxThreads);   // every arithmetic warp gets here
+        if (!*abort_flag) {
+            float* dst = p.energy + (static_cast<size_t>(h) * p.nq + i) * nk;
+            for (int j = static_cast<int>(threadIdx.x) - 64; j < nk; j += kEnergySoftmaxThreads) {
+                float tot = 0.f;
+#pragma unroll
+                for (int w = 0; w < kEnergySoftmaxWarps; ++w) tot += red[w * L::MAX_NK + j];
+                dst[j] = p.accumulate ? dst[j] + tot : tot;
             }
         }
     }
 
+    // ---- teardown (also the abort drain) ----------------------------------------
     __syncthreads();
     if (*abort_flag) {
         constexpr uint64_t kDrainNs = 1000000000ull;
         if (warp == 0 && lane == 0) {
-            if (armed_q) mbar_wait_drain(bar(L::B_Q), 0, kDrainNs);
             for (int s = 0; s < KST; ++s)
                 if (armed_k[s]) mbar_wait_drain(bar(L::B_KF + s), (armed_k[s] - 1) & 1, kDrainNs);
         }

@@ -90,7 +90,8 @@ calib_status calib_device_check(void* stream);
  *              (calib_anchor_rows); then Nq = n_q and blocks are over that sequence.
  *   energy   : fp32 [H, ceil(Nq/B), ceil(N/B)].  accumulate != 0 adds to it (for the
  *              energy-sum aggregation over inputs); 0 overwrites.
- * P is never written to memory. */
+ * P is never written to memory.  N <= 131072 (CALIB_ERR_UNSUPPORTED beyond: the per-block
+ * partial sums of one query block are kept in shared memory). */
 calib_status calib_block_energy(const void* q, const void* k, const float* lse,
                                 int H, int N, int D, int block, float scale,
                                 const int32_t* q_rows, int n_q,

@@ -76,3 +76,6 @@ def test_invalid_arguments_rejected_before_device_work():
     # selection beyond nk = 1024 is unsupported
     assert L.calib_select_mask(fake, 1, 1, 1025, 0.9, null, fake, null, null) in (
         ops.CALIB_ERR_UNSUPPORTED,)
+    # energy pass beyond N = 131072 tokens is unsupported
+    assert L.calib_block_energy(fake, fake, null, 1, 131073, 128, 128, 0.1, null, 0, fake, 0, null) == \
+        ops.CALIB_ERR_UNSUPPORTED
