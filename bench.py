@@ -39,7 +39,7 @@ UNIT = "TFLOPS"
 # DRAM bytes (read + write) of one attn_fwd_kernel launch on the wan13b workload, from an
 # ncu capture (profiles/attn_fwd_wan13b.md), valid only for the kernel sources it was taken
 # on: reported as roofline.traffic while the source hashes still match, else null.
-NCU_TRAFFIC = {("wan13b", "3416fe395751", "a9ea2ee30fca"): 302_676_480 + 86_866_176}
+NCU_TRAFFIC = {("wan13b", "8f96c19d5342", "14017e6adac8"): 303_176_192 + 86_784_000}
 
 # MUFU exp2 throughput of one SM: 4 lanes per clock in each of the 4 sub-partitions.
 MUFU_EX2_PER_CLK_SM = 16
@@ -60,6 +60,20 @@ def _peaks():
                 "hbm_gbs": d["hbm_gbs"], "source": "measured"}
     except (OSError, KeyError, ValueError):
         return {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0, "source": "fallback"}
+
+
+def max_over_ranks(x: float, dist, device) -> float:
+    """The largest value of x over all ranks (every rank gets it): a multi-GPU step time is the
+    slowest rank's device time."""
+    import torch
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tflops(flops_per_rank: float, world: int, ms_max: float) -> float:
+    """Whole-job throughput of `world` replicas that each did `flops_per_rank` in at most ms_max."""
+    return flops_per_rank * world / (ms_max * 1e-3) / 1e12
 
 
 def kept_flops(mask: np.ndarray, N: int, D: int, B: int, repeat_heads=(), n_anchor=None) -> float:
@@ -177,7 +191,7 @@ def run_reference(args):
     for _ in range(args.warmup):
         cpu_baseline(wl, q, k, v, mask, budget_s=0.5)
     for _ in range(args.steps):
-        per_step.append(cpu_baseline(wl, q, k, v, mask, budget_s=max(1.0, 60.0 / max(1, args.steps))))
+        per_step.append(cpu_baseline(wl, q, k, v, mask, budget_s=max(0.5, args.ref_seconds / max(1, args.steps))))
     val = statistics.mean(p["value"] for p in per_step)
     line = {"impl": "reference", "metric": METRIC, "value": val, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
@@ -204,6 +218,69 @@ def run_energy_only(args, wl, dev, torch, ops, synth):
                       "ms": ms, "exp2_per_s": exps, "frac_of_mufu_at_1965mhz": exps / peak}), flush=True)
 
 
+def run_calibration_sweep(dev, torch, ops, synth):
+    """Offline calibration over the sweep workload (12 heads x 32760 tokens, B=128): for each of
+    8 timesteps (positional scale 1 + t/8) and 4 seeded inputs, the fused LSE + energy pass, then
+    the minimal tau-selection for tau in {0.9, 0.95, 0.99} in two aggregation modes -- per-input
+    masks with the cross-input vote (rho = 1/2), and one selection on the energies summed over
+    the inputs (the kernel's accumulate flag).  Reports times, rates and the kept densities."""
+    wl = synth.WORKLOADS["sweep"]
+    s = wl.shape
+    B, N, H, nb = s.block, s.N, s.H, s.nblk
+    n_in, taus, T = wl.extra["n_calib"], wl.extra["taus"], wl.timesteps
+    st = torch.cuda.current_stream()
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    E = torch.empty((H, nb, nb), dtype=torch.float32, device=dev)
+    Esum = torch.empty_like(E)
+    msk = torch.empty((H, nb, nb), dtype=torch.uint8, device=dev)
+    counts = torch.empty((H, nb, nb), dtype=torch.int32, device=dev)
+    dens = {"vote": {str(t_): [] for t_ in taus}, "energy_sum": {str(t_): [] for t_ in taus}}
+    e_ms, a_ms, sel_ms = [], [], []
+    t_start = time.perf_counter()
+    for t in range(T):
+        qk = [synth.make_qkv(wl, input_idx=d, device=dev, pos_scale=1.0 + 0.125 * t)[:2] for d in range(n_in)]
+        ops.block_energy(qk[0][0], qk[0][1], B, out=E)        # warm-up
+        for tau in taus:
+            counts.zero_()
+            for d, (q, k) in enumerate(qk):
+                e0, e1, e2 = ev(), ev(), ev()
+                e0.record(st)
+                ops.block_energy(q, k, B, out=E)
+                e1.record(st)
+                ops.select_mask(E, tau, out=msk, count_accum=counts)
+                e2.record(st)
+                torch.cuda.synchronize()
+                if tau == taus[0]:
+                    e_ms.append(e0.elapsed_time(e1))
+                sel_ms.append(e1.elapsed_time(e2))
+            vote = ops.aggregate_masks(counts, n_in, (1, 2))
+            dens["vote"][str(tau)].append(float(vote.float().mean().item()))
+        for d, (q, k) in enumerate(qk):
+            e0, e1 = ev(), ev()
+            e0.record(st)
+            ops.block_energy(q, k, B, out=Esum, accumulate=d > 0)
+            e1.record(st)
+            torch.cuda.synchronize()
+            a_ms.append(e0.elapsed_time(e1))
+        for tau in taus:
+            dens["energy_sum"][str(tau)].append(float(ops.select_mask(Esum, tau, out=msk).float().mean().item()))
+        del qk
+    ops.device_check()
+    em = statistics.median(e_ms)
+    sm_ = statistics.median(sel_ms)
+    sel_bytes = H * nb * nb * (4 + 1 + 4 + 4)     # energies in, mask out, vote counts read + written
+    exps = 2.0 * N * N * H / (em * 1e-3)
+    peak = MUFU_EX2_PER_CLK_SM * B200_SMS * 1965.0e6
+    print(json.dumps({
+        "leg": "calibration_sweep", "workload": wl.name, "H": H, "N": N, "block": B, "inputs": n_in,
+        "timesteps": T, "taus": list(taus), "energy_passes": len(e_ms) + len(a_ms),
+        "energy_ms_median": em, "energy_exp2_per_s": exps, "energy_frac_of_mufu_at_1965mhz": exps / peak,
+        "energy_tflops_qk": 2 * 2.0 * N * N * s.D * H / (em * 1e-3) / 1e12,
+        "energy_accumulate_ms_median": statistics.median(a_ms),
+        "select_ms_median": sm_, "select_gbs": sel_bytes / (sm_ * 1e-3) / 1e9,
+        "kept_density": dens, "wall_s": time.perf_counter() - t_start}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -217,6 +294,11 @@ def main():
     ap.add_argument("--energy-only", action="store_true",
                     help="time only the fused LSE + block-energy pass (calibration) and print its own line")
     ap.add_argument("--heads", type=int, default=None, help="with --energy-only: the first H heads only")
+    ap.add_argument("--calibration-sweep", action="store_true",
+                    help="the calibration sweep: energies + selection over 4 inputs x 8 timesteps x 3 taus, "
+                         "cross-input vote and energy-sum modes; prints its own line")
+    ap.add_argument("--ref-seconds", type=float, default=60.0,
+                    help="--impl reference: total seconds of oracle work over the timed steps")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -242,6 +324,8 @@ def main():
     B, D, N, H = s.block, s.D, s.N, s.H
     if args.energy_only:
         return run_energy_only(args, wl, dev, torch, ops, synth)
+    if args.calibration_sweep:
+        return run_calibration_sweep(dev, torch, ops, synth)
     q, k, v = synth.make_qkv(wl, device=dev)
     mask_np = synth.make_head_masks(wl, timestep=args.timestep)
     mask = torch.from_numpy(mask_np).to(dev)
@@ -281,10 +365,8 @@ def main():
     ops.device_check()
     ms = e0.elapsed_time(e1) / args.steps
     if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
-    value = flops_kept * world / (ms * 1e-3) / 1e12
+        ms = max_over_ranks(ms, dist, dev)
+    value = whole_job_tflops(flops_kept, world, ms)
     peaks = _peaks()
 
     extras = {}
@@ -330,9 +412,7 @@ def main():
 
         ms_e2e = _time_calls(e2e_step, 10, 3, torch)
         if world > 1:
-            t = torch.tensor([ms_e2e], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ms_e2e = float(t.item())
+            ms_e2e = max_over_ranks(ms_e2e, dist, dev)
         nb = q.numel() * q.element_size()
         extras["e2e"] = {"value": flops_kept * world / (ms_e2e * 1e-3) / 1e12, "unit": UNIT,
                          "h2d_bytes_per_step": 3 * nb, "d2h_bytes_per_step": nb, "ms_per_step": ms_e2e}

@@ -96,22 +96,21 @@ calib_status launch_status() {
 
 // ---- attention ---------------------------------------------------------------------
 template <int D, int BLK, bool WITH_LSE>
-calib_status launch_attn(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+calib_status launch_attn(const CUtensorMap& tk, const CUtensorMap& tv,
                          const calib::AttnParams& p, int grid, cudaStream_t st) {
     constexpr int KST = 3, VST = 3;   // K / V ring depths
     using L = calib::AttnSmem<D, BLK, KST, VST>;
     static_assert(L::BYTES <= 232448, "shared memory budget");
     auto* fn = calib::attn_fwd_kernel<D, BLK, KST, VST, WITH_LSE>;
     if (calib_status s = ensure_smem(reinterpret_cast<const void*>(fn), L::BYTES)) return s;
-    fn<<<grid, calib::kAttnThreads, L::BYTES, st>>>(tq, tk, tv, p);
+    fn<<<grid, calib::kAttnThreads, L::BYTES, st>>>(tk, tv, p);
     return launch_status();
 }
 
 template <int D, int BLK>
-calib_status launch_attn_lse(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+calib_status launch_attn_lse(const CUtensorMap& tk, const CUtensorMap& tv,
                              const calib::AttnParams& p, int grid, cudaStream_t st) {
-    return p.lse ? launch_attn<D, BLK, true>(tq, tk, tv, p, grid, st)
-                 : launch_attn<D, BLK, false>(tq, tk, tv, p, grid, st);
+    return p.lse ? launch_attn<D, BLK, true>(tk, tv, p, grid, st) : launch_attn<D, BLK, false>(tk, tv, p, grid, st);
 }
 
 calib_status attn_common(const void* q, const void* k, const void* v, void* o, float* lse, int H, int N,
@@ -150,15 +149,12 @@ calib_status attn_common(const void* q, const void* k, const void* v, void* o, f
     p.out_f32 = (flags & CALIB_ATTN_OUT_F32) ? 1 : 0;
     p.timeout_ns = kDefaultTimeoutNs;
 
-    CUtensorMap tq, tk, tv;
-    if (!make_tmap(&tq, q, D, N, H, calib::kTileM) || !make_tmap(&tk, k, D, N, H, B) ||
-        !make_tmap(&tv, v, D, N, H, B))
-        return CALIB_ERR_CUDA;
+    CUtensorMap tk, tv;
+    if (!make_tmap(&tk, k, D, N, H, B) || !make_tmap(&tv, v, D, N, H, B)) return CALIB_ERR_CUDA;
     cudaStream_t st = as_stream(stream);
-    if (D == 128) return B == 128 ? launch_attn_lse<128, 128>(tq, tk, tv, p, grid, st)
-                                  : launch_attn_lse<128, 64>(tq, tk, tv, p, grid, st);
-    return B == 128 ? launch_attn_lse<64, 128>(tq, tk, tv, p, grid, st)
-                    : launch_attn_lse<64, 64>(tq, tk, tv, p, grid, st);
+    if (D == 128) return B == 128 ? launch_attn_lse<128, 128>(tk, tv, p, grid, st)
+                                  : launch_attn_lse<128, 64>(tk, tv, p, grid, st);
+    return B == 128 ? launch_attn_lse<64, 128>(tk, tv, p, grid, st) : launch_attn_lse<64, 64>(tk, tv, p, grid, st);
 }
 
 // ---- energy ------------------------------------------------------------------------

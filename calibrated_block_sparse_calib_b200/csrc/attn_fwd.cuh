@@ -8,29 +8,34 @@
 // broadcast to the other rows of their frame ([zh] §2.2B, [fr] §2.C).
 //
 // One CTA per work item (head h, query block i).  320 threads:
-//   warp 0      TMA producer: Q tile once (repeat heads: nothing, their anchor rows are
-//               gathered by the softmax warps), then K_j / V_j for each kept j through
-//               KST / VST-deep rings (K runs one tile ahead of V).
+//   warp 0      TMA producer: K_j / V_j for each kept j through KST / VST-deep rings (K
+//               runs one tile ahead of V).
 //   warp 1      TMEM owner (512 columns) and MMA issuer (one elected lane of the
 //               converged warp):
-//               S_t = Q K_j^T           SS MMA, M=128, N=B, K=D, into S buffer t%2;
+//               S_t = Q K_j^T           TS MMA, M=128, N=B, K=D: Q from TMEM, K from SMEM;
 //               O_h += P_t,h V_j,h      TS MMA, M=128, N=D, K=B/2, for the two column
 //                                       halves h of the tile: P from TMEM, V from SMEM.
-//   warps 2..9  softmax + epilogue.  Each query row (TMEM lane) is split between two
-//               warps: warps 2..5 own the first half of every key tile's columns, warps
-//               6..9 the second half.  The two halves run INDEPENDENT online-softmax
-//               chains (own running max m_h, own row sum l_h, own accumulator O_h), so
-//               no per-tile exchange couples them; the epilogue merges them once:
+//               Q lives in tensor memory, so QK reads only K from shared memory (with Q in
+//               shared memory too, the operand reads, not the math, set the MMA rate).
+//   warps 2..9  softmax + epilogue.  Warps 2..5 first write the Q tile into tensor memory
+//               (contiguous rows, or the gathered anchor rows of a repeat head).  Each query
+//               row (TMEM lane) is split between two warps: warps 2..5 own the first half of
+//               every key tile's columns, warps 6..9 the second half.  The two halves run
+//               INDEPENDENT online-softmax chains (own running max m_h, own row sum l_h, own
+//               accumulator O_h), so no per-tile exchange couples them; the epilogue merges
+//               them once:
 //               O = (O_0 2^(m_0-m) + O_1 2^(m_1-m)) / (l_0 2^(m_0-m) + l_1 2^(m_1-m)).
-//               Per tile a thread loads its B/2 logits, takes the row max in the log2
-//               domain with lazy rescaling (O_h is rescaled only when m_h grows by more
-//               than 2^8), writes P = 2^(x - m_h) back over its own S columns as bf16 and
-//               adds the bf16-ROUNDED P into l_h, so the normaliser is exactly the sum of
-//               the weights that entered the PV product.
+//               Per tile a thread loads its B/2 logits and hands S back at once (so QK_{t+1}
+//               overlaps this tile's softmax), takes the row max in the log2 domain with
+//               lazy rescaling (O_h is rescaled only when m_h grows by more than 2^8),
+//               writes P = 2^(x - m_h) as bf16 into the P region once PV_{t-1} has consumed
+//               the previous P, and adds the bf16-ROUNDED P into l_h, so the normaliser is
+//               exactly the sum of the weights that entered the PV product.
 // Each row's key list is walked starting at its diagonal block (the first kept key block
 // at or after the query block), where local attention peaks, so the running max is
 // usually final after the first tile and O is rarely rescaled.
-// Tensor memory: S0 = cols [0,128), S1 = [128,256), O_0 = [256, 256+D), O_1 = [256+D, 256+2D).
+// Tensor memory: S = cols [0,128), P = [128,192) (P_0 then P_1, packed bf16 pairs),
+// Q = [192, 192+D/2), O_0 = [256, 256+D), O_1 = [256+D, 256+2D).
 #pragma once
 #include <cuda_bf16.h>
 #include "ptx.cuh"
@@ -42,11 +47,14 @@ constexpr int kSoftmaxThreads = 256;      // warps 2..9
 constexpr int kTileM = 128;               // query rows per tile (MMA M)
 constexpr float kRescaleLog2 = 8.0f;      // rescale O only when the row max grows by > 2^8
 constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kTmemS = 0;            // S tile (fp32, B columns)
+constexpr uint32_t kTmemP = 128;          // P tile (bf16 pairs, B/2 columns: half 0 then half 1)
+constexpr uint32_t kTmemQ = 192;          // Q tile (bf16 pairs, D/2 columns)
 constexpr uint32_t kTmemO = 256;          // first column of O_0 (O_1 follows at kTmemO + D)
 constexpr uint32_t kBarSoftmax = 1;       // named barrier of the softmax warps
 
 struct AttnParams {
-    const __nv_bfloat16* q;   // [H, N, D] (read directly only for repeat-head gathers)
+    const __nv_bfloat16* q;   // [H, N, D]
     __nv_bfloat16* o;         // [H, N, D], bf16 (or fp32 when out_f32)
     float* lse;               // [H, N] or nullptr
     const int32_t* row_ptr;   // [H*nq + 1]
@@ -76,19 +84,6 @@ __device__ __forceinline__ int anchor_token(const AttnParams& p, int a) {
     return p.F * p.Hl * p.Wl + (a - nva);
 }
 
-// Gather one 128-byte-swizzled Q row (D bf16) from global memory into the tile.
-template <int D>
-__device__ __forceinline__ void gather_q_row(uint8_t* sQ, int r, const __nv_bfloat16* src) {
-#pragma unroll
-    for (int c16 = 0; c16 < D / 8; ++c16) {
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (src) v = __ldg(reinterpret_cast<const uint4*>(src) + c16);
-        const int atom = c16 >> 3, chunk = c16 & 7;
-        uint8_t* dst = sQ + atom * (kTileM * 128) + r * 128 + ((chunk ^ (r & 7)) << 4);
-        *reinterpret_cast<uint4*>(dst) = v;
-    }
-}
-
 // Write 32 output values of one row (already normalised).
 __device__ __forceinline__ void store_row32_bf16(__nv_bfloat16* dst, const uint32_t (&packed)[16]) {
     uint4* d = reinterpret_cast<uint4*>(dst);
@@ -106,19 +101,18 @@ template <int D, int BLK, int KST, int VST>
 struct AttnSmem {
     static constexpr int CH = D / 64;                     // 128-byte chunks per row
     static constexpr uint32_t CHUNK = BLK * 128;          // one 64-column chunk of a K/V tile
-    static constexpr uint32_t Q_BYTES = CH * kTileM * 128;
     static constexpr uint32_t K_BYTES = CH * CHUNK;
-    static constexpr uint32_t OFF_K = Q_BYTES;
+    static constexpr uint32_t OFF_K = 0;
     static constexpr uint32_t OFF_V = OFF_K + KST * K_BYTES;
     static constexpr uint32_t OFF_BAR = OFF_V + VST * K_BYTES;
     // barrier indices
     static constexpr int B_Q = 0, B_KF = 1, B_KE = B_KF + KST, B_VF = B_KE + KST,
-                         B_VE = B_VF + VST, B_SF = B_VE + VST, B_PF = B_SF + 2, B_O = B_PF + 2,
-                         B_DRAIN = B_O + 1, NBARS = B_DRAIN + 1;
+                         B_VE = B_VF + VST, B_SF = B_VE + VST, B_SE = B_SF + 1, B_PF = B_SE + 1,
+                         B_O = B_PF + 1, B_DRAIN = B_O + 1, NBARS = B_DRAIN + 1;
     static constexpr uint32_t OFF_MISC = OFF_BAR + NBARS * 8;   // tmem base, abort flag, t0
     // The epilogue's exchange of (m, l) between the two halves of a row, float4 [2][128],
-    // reuses the Q tile: by then every MMA that read Q has completed.
-    static constexpr uint32_t OFF_XCH = 0;
+    // reuses the first K stage: by then every MMA that read it has completed.
+    static constexpr uint32_t OFF_XCH = OFF_K;
     // + alignment slack; at least 120 KB so that one CTA (holding all 512 TMEM columns)
     // is resident per SM and no CTA waits in tcgen05.alloc.
     static constexpr uint32_t RAW = OFF_MISC + 16 + 1024;
@@ -127,15 +121,14 @@ struct AttnSmem {
 
 template <int D, int BLK, int KST, int VST, bool WITH_LSE>
 __global__ void __launch_bounds__(kAttnThreads, 1)
-attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
+attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                const AttnParams p) {
     using L = AttnSmem<D, BLK, KST, VST>;
     constexpr int CH = L::CH;
     constexpr int HC = BLK / 2;                            // key columns per softmax half
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
-    uint8_t* sQ = smem;
     uint8_t* sK = smem + L::OFF_K;
     uint8_t* sV = smem + L::OFF_V;
     const uint32_t bar0 = smem_u32(smem + L::OFF_BAR);
@@ -165,11 +158,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
     // ---- setup ------------------------------------------------------------------
     if (threadIdx.x == 0) {
-        mbar_init(bar(L::B_Q), rep ? 128u : 1u);
+        mbar_init(bar(L::B_Q), 128u);
         for (int s = 0; s < KST; ++s) { mbar_init(bar(L::B_KF + s), 1); mbar_init(bar(L::B_KE + s), 1); }
         for (int s = 0; s < VST; ++s) { mbar_init(bar(L::B_VF + s), 1); mbar_init(bar(L::B_VE + s), 1); }
-        for (int b = 0; b < 2; ++b) mbar_init(bar(L::B_SF + b), 1);
-        for (int b = 0; b < 2; ++b) mbar_init(bar(L::B_PF + b), kSoftmaxThreads);
+        mbar_init(bar(L::B_SF), 1);
+        mbar_init(bar(L::B_SE), kSoftmaxThreads);
+        mbar_init(bar(L::B_PF), kSoftmaxThreads);
         mbar_init(bar(L::B_O), 1);
         mbar_init(bar(L::B_DRAIN), 1);
         *abort_flag = 0;
@@ -183,7 +177,6 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         fence_barrier_init();
     }
     if (warp == 0 && lane == 0) {
-        tma_prefetch_desc(&tm_q);
         tma_prefetch_desc(&tm_k);
         tma_prefetch_desc(&tm_v);
     }
@@ -204,7 +197,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     };
 
     // bookkeeping for the abort drain (producer only)
-    int armed_q = 0, armed_k[KST], armed_v[VST];
+    int armed_k[KST], armed_v[VST];
 #pragma unroll
     for (int s = 0; s < KST; ++s) armed_k[s] = 0;
 #pragma unroll
@@ -213,14 +206,6 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     if (warp == 0) {
         // ===================== TMA producer (converged warp, one elected lane issues) ====
         if (nkept > 0) {
-            if (!rep) {
-                if (elect_one()) {
-                    mbar_arrive_expect_tx(bar(L::B_Q), L::Q_BYTES);
-                    for (int c = 0; c < CH; ++c)
-                        tma_load_3d(smem_u32(sQ + c * kTileM * 128), &tm_q, bar(L::B_Q), c * 64, i * BLK, h);
-                }
-                armed_q = 1;
-            }
             auto issue_k = [&](int t) -> bool {
                 const int s = t % KST;
                 if (!mbar_wait_warp(bar(L::B_KE + s), ((t / KST) & 1) ^ 1, ctl)) return false;
@@ -258,27 +243,40 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         if (nkept > 0) {
             constexpr uint32_t idesc_qk = idesc_bf16_f32(kTileM, BLK, false, false);
             constexpr uint32_t idesc_pv = idesc_bf16_f32(kTileM, D, false, true);
-            const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV);
-            bool ok = mbar_wait_warp(bar(L::B_Q), 0, ctl);
+            const uint32_t sKa = smem_u32(sK), sVa = smem_u32(sV);
+            bool ok = mbar_wait_warp(bar(L::B_Q), 0, ctl);   // Q written into tensor memory
             tc_fence_after();
             // Every tcgen05.mma blocks its issuer while the tensor pipe's short queue is
-            // full, so any time this warp spends between MMA batches leaves the pipe idle.
-            // The loop has two wait points per tile, both normally already satisfied: the
-            // K/V tiles (loaded ahead) before QK, and P before PV.  Each wait's first
-            // try_wait is issued before the preceding MMA batch, so its latency (an mbarrier
-            // round trip, ~100 cycles) overlaps that batch's issue.
+            // full, so time this warp spends between MMA batches leaves the pipe idle.  Per
+            // tile there are two wait points, normally already satisfied when reached: S
+            // handed back (and K loaded) before QK_{t+1}, and P (and V) before PV_t.  Each
+            // wait's first try_wait is issued before the preceding MMA batch, so its
+            // latency overlaps that batch.
             auto qk = [&](int t) {
                 const int s = t % KST;
-                const uint32_t d_tmem = tmem + (t & 1) * 128;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t inner = (kk & 3) * 32;   // K step of 16 bf16 inside a 128-B atom
-                    const uint64_t ad = smem_desc_sw128(sQa + (kk >> 2) * kTileM * 128 + inner, 16, 1024);
-                    const uint64_t bd = smem_desc_sw128(sKa + s * L::K_BYTES + (kk >> 2) * L::CHUNK + inner, 16, 1024);
-                    umma_ss(d_tmem, ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
+                    const uint64_t bd =
+                        smem_desc_sw128(sKa + s * L::K_BYTES + (kk >> 2) * L::CHUNK + (kk & 3) * 32, 16, 1024);
+                    umma_ts(tmem + kTmemS, tmem + kTmemQ + kk * 8, bd, idesc_qk, kk > 0 ? 1u : 0u);
                 }
-                umma_commit(bar(L::B_SF + (t & 1)));
+                umma_commit(bar(L::B_SF));
                 umma_commit(bar(L::B_KE + s));
+            };
+            auto pv = [&](int t) {
+                const int sv = t % VST;
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf) {
+#pragma unroll
+                    for (int kk = 0; kk < HC / 16; ++kk) {
+                        const uint64_t bd =
+                            smem_desc_sw128(sVa + sv * L::K_BYTES + (hf * HC + kk * 16) * 128, L::CHUNK, 1024);
+                        umma_ts(tmem + kTmemO + hf * D, tmem + kTmemP + hf * (HC / 2) + kk * 8, bd, idesc_pv,
+                                (t > 0 || kk > 0) ? 1u : 0u);
+                    }
+                }
+                umma_commit(bar(L::B_O));
+                umma_commit(bar(L::B_VE + sv));
             };
             auto kf = [&](int t) { return bar(L::B_KF + t % KST); };
             auto kf_par = [&](int t) -> uint32_t { return (t / KST) & 1; };
@@ -289,41 +287,22 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 tc_fence_after();
                 if (elect_one()) qk(0);
             }
-            bool tok_k = nkept > 1 ? mbar_try_wait(kf(1), kf_par(1)) : true;
-            bool tok_v = mbar_try_wait(vf(0), vf_par(0));
             for (int t = 0; ok && t < nkept; ++t) {
-                const int sv = t % VST;
-                if (t + 1 < nkept) ok = mbar_wait_warp_tok(kf(t + 1), kf_par(t + 1), tok_k, ctl);
-                if (ok) ok = mbar_wait_warp_tok(vf(t), vf_par(t), tok_v, ctl);
-                if (!ok) break;
-                tc_fence_after();
-                const bool tok_p = mbar_try_wait(bar(L::B_PF + (t & 1)), (t >> 1) & 1);
-                // S buffer (t+1)&1 last held P_{t-1}, the A operand of PV_{t-1}.  This thread
-                // issued PV_{t-1} before this QK, and tcgen05.mma operations of one issuing
-                // thread execute in issue order, so QK_{t+1} overwrites the buffer only after
-                // PV_{t-1} has read it: no completion wait.
-                if (t + 1 < nkept && elect_one()) qk(t + 1);
-                ok = mbar_wait_warp_tok(bar(L::B_PF + (t & 1)), (t >> 1) & 1, tok_p, ctl);
-                if (!ok) break;
-                tc_fence_after();
-                tok_k = t + 2 < nkept ? mbar_try_wait(kf(t + 2), kf_par(t + 2)) : true;
-                tok_v = t + 1 < nkept ? mbar_try_wait(vf(t + 1), vf_par(t + 1)) : true;
-                if (elect_one()) {
-                    // O_h += P_t,h V_j,h for both column halves; P_t,h is packed bf16 in the
-                    // first HC/2 columns of the half's S columns
-#pragma unroll
-                    for (int hf = 0; hf < 2; ++hf) {
-#pragma unroll
-                        for (int kk = 0; kk < HC / 16; ++kk) {
-                            const uint64_t bd =
-                                smem_desc_sw128(sVa + sv * L::K_BYTES + (hf * HC + kk * 16) * 128, L::CHUNK, 1024);
-                            umma_ts(tmem + kTmemO + hf * D, tmem + (t & 1) * 128 + hf * HC + kk * 8, bd, idesc_pv,
-                                    (t > 0 || kk > 0) ? 1u : 0u);
-                        }
-                    }
-                    umma_commit(bar(L::B_O));
-                    umma_commit(bar(L::B_VE + sv));
+                if (t + 1 < nkept) {
+                    // QK_{t+1} overwrites S once every softmax thread has loaded S_t
+                    const bool tok_s = mbar_test(bar(L::B_SE), t & 1);
+                    ok = mbar_wait_warp(kf(t + 1), kf_par(t + 1), ctl);
+                    if (ok) ok = mbar_wait_warp_tok(bar(L::B_SE), t & 1, tok_s, ctl);
+                    if (!ok) break;
+                    tc_fence_after();
+                    if (elect_one()) qk(t + 1);
                 }
+                const bool tok_p = mbar_test(bar(L::B_PF), t & 1);
+                ok = mbar_wait_warp(vf(t), vf_par(t), ctl);
+                if (ok) ok = mbar_wait_warp_tok(bar(L::B_PF), t & 1, tok_p, ctl);
+                if (!ok) break;
+                tc_fence_after();
+                if (elect_one()) pv(t);
             }
         }
     } else {
@@ -333,12 +312,29 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const int r = static_cast<int>(q4 * 32 + lane);   // tile row == TMEM lane
         const uint32_t lane_base = (q4 * 32) << 16;
         const uint32_t o_col = kTmemO + hf * D;            // this half's accumulator O_h
-        if (rep && nkept > 0 && hf == 0) {
+        if (nkept > 0 && hf == 0) {
+            // Q row -> tensor memory: the bf16 pairs of the row in memory order are the
+            // packed TS operand.  Rows past the block or the sequence are zero.
             const int a = i * BLK + r;
-            const __nv_bfloat16* src =
-                (a < Nq) ? p.q + (static_cast<size_t>(h) * p.N + anchor_token(p, a)) * D : nullptr;
-            gather_q_row<D>(sQ, r, src);
-            fence_proxy_async_smem();
+            const uint4* src = (r < BLK && a < Nq)
+                                   ? reinterpret_cast<const uint4*>(
+                                         p.q + (static_cast<size_t>(h) * p.N + (rep ? anchor_token(p, a) : a)) * D)
+                                   : nullptr;
+            uint32_t w[32];
+#pragma unroll
+            for (int c = 0; c < D / 64; ++c) {
+#pragma unroll
+                for (int v = 0; v < 8; ++v) {
+                    const uint4 x = src ? __ldg(src + c * 8 + v) : make_uint4(0, 0, 0, 0);
+                    w[4 * v] = x.x;
+                    w[4 * v + 1] = x.y;
+                    w[4 * v + 2] = x.z;
+                    w[4 * v + 3] = x.w;
+                }
+                tmem_st32(tmem + lane_base + kTmemQ + c * 32, w);
+            }
+            tmem_wait_st();
+            tc_fence_before();
             mbar_arrive(bar(L::B_Q));
         }
         const float sc = p.scale_log2;
@@ -349,18 +345,19 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         for (int t = 0; t < nkept; ++t) {
             const int j = p.col_idx[kidx(t)];
             const int valid = min(BLK, p.N - j * BLK) - hf * HC;   // may be <= 0 (ragged tail)
-            ok = mbar_wait_warp(bar(L::B_SF + (t & 1)), (t >> 1) & 1, ctl);
+            ok = mbar_wait_warp(bar(L::B_SF), t & 1, ctl);
             if (!ok) break;
             tc_fence_after();
-            const uint32_t s_col = (t & 1) * 128 + hf * HC;
             float s[HC];
             {
                 uint32_t raw[HC];
-                if constexpr (HC == 64) tmem_ld64_wait(tmem + lane_base + s_col, raw);
-                else tmem_ld32_wait(tmem + lane_base + s_col, raw);
+                if constexpr (HC == 64) tmem_ld64_wait(tmem + lane_base + kTmemS + hf * HC, raw);
+                else tmem_ld32_wait(tmem + lane_base + kTmemS + hf * HC, raw);
 #pragma unroll
                 for (int c = 0; c < HC; ++c) s[c] = __uint_as_float(raw[c]);
             }
+            tc_fence_before();
+            mbar_arrive(bar(L::B_SE));                 // S may be overwritten by QK_{t+1} now
             if (valid < HC) {                       // ragged last key block only
 #pragma unroll
                 for (int c = 0; c < HC; ++c)
@@ -406,19 +403,20 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             l_run = l_run * alpha + ((lr0 + lr1) + (lr2 + lr3));
             if constexpr (WITH_LSE) l_ex = l_ex * alpha + (le0 + le1);
             m_run = m_new;
-            if constexpr (HC == 64) tmem_st32(tmem + lane_base + s_col, *reinterpret_cast<const uint32_t(*)[32]>(pk));
-            else tmem_st16(tmem + lane_base + s_col, pk);
-            // Consume the completion of PV_{t-1} (both halves) on every tile.  An mbarrier
-            // parity wait is only unambiguous while the waiter is at most one phase behind;
-            // waiting on every phase keeps it so (PV_t cannot start before this P is ready),
-            // and by now PV_{t-1} has normally finished.
+            // P_{t-1}, in the same columns, is the operand of PV_{t-1}; O is rescaled below.
+            // Consume the completion of PV_{t-1} on every tile: an mbarrier parity wait is only
+            // unambiguous while the waiter is at most one phase behind, and PV_t cannot start
+            // before this P is ready.
             if (t > 0) {
                 ok = mbar_wait_warp(bar(L::B_O), (t - 1) & 1, ctl);
                 if (!ok) break;
+                tc_fence_after();
             }
+            const uint32_t p_col = kTmemP + hf * (HC / 2);
+            if constexpr (HC == 64) tmem_st32(tmem + lane_base + p_col, *reinterpret_cast<const uint32_t(*)[32]>(pk));
+            else tmem_st16(tmem + lane_base + p_col, pk);
             if (__any_sync(0xffffffffu, upd && t > 0)) {
                 // rescale O_h, accumulated through PV_{t-1}, in place
-                tc_fence_after();
                 const float a_row = (upd && t > 0) ? alpha : 1.f;
                 uint32_t raw[32];
 #pragma unroll
@@ -431,7 +429,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(bar(L::B_PF + (t & 1)));
+            mbar_arrive(bar(L::B_PF));
         }
         // completion of the last PV (the loop consumed every earlier one)
         if (ok && nkept > 0) ok = mbar_wait_warp(bar(L::B_O), (nkept - 1) & 1, ctl);
@@ -523,7 +521,6 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     if (*abort_flag) {
         constexpr uint64_t kDrainNs = 1000000000ull;
         if (warp == 0 && lane == 0) {
-            if (armed_q) mbar_wait_drain(bar(L::B_Q), 0, kDrainNs);
             for (int s = 0; s < KST; ++s)
                 if (armed_k[s]) mbar_wait_drain(bar(L::B_KF + s), (armed_k[s] - 1) & 1, kDrainNs);
             for (int s = 0; s < VST; ++s)

@@ -118,7 +118,7 @@ __device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, co
     return __all_sync(0xffffffffu, ok);
 }
 
-// Second half of a split wait: `tok` is each lane's mbar_try_wait result for the same
+// Second half of a split wait: `tok` is each lane's mbar_test result for the same
 // phase, issued earlier so that its latency overlapped other work.  The phase being waited
 // for must be the barrier's current or next one (never two phases ahead of the last one
 // this warp consumed), or the parity test would be ambiguous.
