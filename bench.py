@@ -423,6 +423,12 @@ def main():
             msk = torch.empty(energy.shape, dtype=torch.uint8, device=dev)
             ms_sel = _time_calls(lambda: ops.select_mask(energy, 0.95, out=msk), 20, 3, torch)
             sel_bytes = energy.numel() * 4 + msk.numel()
+            # LSE reuse: a dense forward that emits the row LSE (calibration runs the dense
+            # model anyway), then the energy pass with that LSE runs a single pass
+            lse_buf = torch.empty((H, N), dtype=torch.float32, device=dev)
+            ms_attn_lse = _time_calls(lambda: ops.sparse_attn_fwd(q, k, v, bl_dense, out=out, lse=lse_buf),
+                                      5, 2, torch)
+            ms_e1 = _time_calls(lambda: ops.block_energy(q, k, B, lse=lse_buf, out=energy), 5, 2, torch)
             exps = 2.0 * N * N * H / (ms_energy * 1e-3)
             clk_mhz = (clk.summary().get("sm_max_mhz") or 1965.0)
             mufu_peak = MUFU_EX2_PER_CLK_SM * B200_SMS * clk_mhz * 1e6
@@ -430,12 +436,25 @@ def main():
                 "energy_ms": ms_energy,
                 "energy_tflops_qk": 2 * 2.0 * N * N * D * H / (ms_energy * 1e-3) / 1e12,
                 "energy_exps_per_s": exps,
+                "energy_with_attention_lse": {"dense_fwd_with_lse_ms": ms_attn_lse, "energy_one_pass_ms": ms_e1,
+                                              "exp2_per_s": N * N * H / (ms_e1 * 1e-3)},
                 "energy_roofline": {"bound": "alu", "unit": "exp2/s", "achieved": exps, "peak": mufu_peak,
                                     "frac": exps / mufu_peak, "kernel": f"block_energy_kernel<{D},{B},4>",
                                     "peak_source": "16 MUFU ex2 per clock per SM x 148 SMs x max SM clock"},
                 "select_ms": ms_sel, "select_gbs": sel_bytes / (ms_sel * 1e-3) / 1e9,
                 "select_frac_hbm": sel_bytes / (ms_sel * 1e-3) / 1e9 / peaks["hbm_gbs"],
                 "tau": 0.95, "selected_density": float(msk.float().mean().item())}
+            # interval form of the default workload's skip list (mask storage)
+            rows = H * s.nblk
+            iv = ops.csr_to_intervals(bl.row_ptr, bl.col_idx, H, s.nblk)
+            ms_enc = _time_calls(lambda: ops.lib().calib_csr_to_intervals(
+                bl.row_ptr.data_ptr(), bl.col_idx.data_ptr(), H, s.nblk, iv[0].data_ptr(),
+                iv[1].data_ptr(), iv[2].data_ptr(), None), 20, 3, torch)
+            nnz, n_iv = int(bl.row_ptr[-1].item()), int(iv[0][-1].item())
+            extras["calibration"]["skip_list_intervals"] = {
+                "kept_blocks": nnz, "runs": n_iv, "blocks_per_run": nnz / max(1, n_iv),
+                "csr_bytes": 4 * (rows + 1) + 2 * nnz, "interval_bytes": 4 * (rows + 1) + 4 * n_iv,
+                "encode_ms": ms_enc}
             ops.device_check()
 
     line = {

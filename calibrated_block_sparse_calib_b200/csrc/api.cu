@@ -17,6 +17,7 @@
 #include "attn_fwd.cuh"
 #include "energy.cuh"
 #include "select.cuh"
+#include "intervals.cuh"
 
 namespace {
 
@@ -266,6 +267,35 @@ calib_status calib_mask_to_csr(const uint8_t* mask, int H, int nq, int nk, int32
     calib::csr_count_kernel<<<rows_grid(rows), 128, 0, st>>>(mask, rows, nk, row_ptr_out);
     calib::csr_scan_kernel<<<1, 1024, 0, st>>>(row_ptr_out, rows);
     calib::csr_fill_kernel<<<rows_grid(rows), 128, 0, st>>>(mask, rows, nk, row_ptr_out, col_idx_out);
+    return launch_status();
+}
+
+calib_status calib_csr_to_intervals(const int32_t* row_ptr, const int16_t* col_idx, int H, int nq,
+                                    int32_t* iv_ptr_out, int16_t* iv_start_out, int16_t* iv_len_out, void* stream) {
+    if (!row_ptr || !col_idx || !iv_ptr_out || !iv_start_out || !iv_len_out) return CALIB_ERR_INVALID;
+    if (H < 1 || nq < 1 || static_cast<long long>(H) * nq > (1ll << 31) - 2) return CALIB_ERR_INVALID;
+    if (calib_status s = check_device()) return s;
+    const int rows = H * nq;
+    cudaStream_t st = as_stream(stream);
+    calib::iv_count_kernel<<<rows_grid(rows), 128, 0, st>>>(row_ptr, col_idx, rows, iv_ptr_out);
+    calib::csr_scan_kernel<<<1, 1024, 0, st>>>(iv_ptr_out, rows);
+    calib::iv_fill_kernel<<<rows_grid(rows), 128, 0, st>>>(row_ptr, col_idx, rows, iv_ptr_out, iv_start_out,
+                                                           iv_len_out);
+    return launch_status();
+}
+
+calib_status calib_intervals_to_csr(const int32_t* iv_ptr, const int16_t* iv_start, const int16_t* iv_len, int H,
+                                    int nq, int32_t* row_ptr_out, int16_t* col_idx_out, void* stream) {
+    if (!iv_ptr || !iv_start || !iv_len || !row_ptr_out) return CALIB_ERR_INVALID;
+    if (H < 1 || nq < 1 || static_cast<long long>(H) * nq > (1ll << 31) - 2) return CALIB_ERR_INVALID;
+    if (calib_status s = check_device()) return s;
+    const int rows = H * nq;
+    cudaStream_t st = as_stream(stream);
+    calib::iv_total_kernel<<<rows_grid(rows), 128, 0, st>>>(iv_ptr, iv_len, rows, row_ptr_out);
+    calib::csr_scan_kernel<<<1, 1024, 0, st>>>(row_ptr_out, rows);
+    if (col_idx_out)
+        calib::iv_expand_kernel<<<rows_grid(rows), 128, 0, st>>>(iv_ptr, iv_start, iv_len, rows, row_ptr_out,
+                                                                 col_idx_out);
     return launch_status();
 }
 

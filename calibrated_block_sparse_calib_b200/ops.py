@@ -44,6 +44,8 @@ _SIGS = {
     "calib_aggregate_masks": ([_P, _I, _I, _I, _I, _I, _I, _P, _P], ctypes.c_int),
     "calib_mask_to_csr": ([_P, _I, _I, _I, _P, _P, _P], ctypes.c_int),
     "calib_build_schedule": ([_P, _I, _I, _P, _P], ctypes.c_int),
+    "calib_csr_to_intervals": ([_P, _P, _I, _I, _P, _P, _P, _P], ctypes.c_int),
+    "calib_intervals_to_csr": ([_P, _P, _P, _I, _I, _P, _P, _P], ctypes.c_int),
     "calib_anchor_count": ([_I, _I, _I, _I, _I], ctypes.c_int64),
     "calib_anchor_rows": ([_I, _I, _I, _I, _I, _P, _P], ctypes.c_int),
     "sparse_attn_fwd": ([_P, _P, _P, _P, _P, _I, _I, _I, _F, ctypes.POINTER(_BlockListC), _U32, _P],
@@ -178,6 +180,41 @@ def mask_to_csr(mask: torch.Tensor):
     _check("calib_mask_to_csr", lib().calib_mask_to_csr(
         _ptr(mask), H, nq, nk, _ptr(row_ptr), _ptr(col_idx), _stream()))
     return row_ptr, col_idx
+
+
+def csr_to_intervals(row_ptr: torch.Tensor, col_idx: torch.Tensor, H: int, nq: int):
+    """Runs of consecutive kept blocks per row: (iv_ptr int32 [H*nq+1], starts int16, lengths
+    int16), the runs trimmed to their count."""
+    _need(row_ptr, "row_ptr", torch.int32, (H * nq + 1,))
+    _need(col_idx, "col_idx", torch.int16)
+    cap = max(1, col_idx.numel())
+    iv_ptr = torch.empty(H * nq + 1, dtype=torch.int32, device=row_ptr.device)
+    starts = torch.empty(cap, dtype=torch.int16, device=row_ptr.device)
+    lens = torch.empty(cap, dtype=torch.int16, device=row_ptr.device)
+    _check("calib_csr_to_intervals", lib().calib_csr_to_intervals(
+        _ptr(row_ptr), _ptr(col_idx), H, nq, _ptr(iv_ptr), _ptr(starts), _ptr(lens), _stream()))
+    n = int(iv_ptr[-1].item())
+    return iv_ptr, starts[:n], lens[:n]
+
+
+def intervals_to_csr(iv_ptr: torch.Tensor, starts: torch.Tensor, lens: torch.Tensor, H: int, nq: int):
+    """CSR skip list (row_ptr int32 [H*nq+1], col_idx int16 [nnz]) from runs: one call
+    sizes the list (row_ptr only), the second fills it."""
+    _need(iv_ptr, "iv_ptr", torch.int32, (H * nq + 1,))
+    _need(starts, "starts", torch.int16)
+    _need(lens, "lens", torch.int16, starts.shape)
+    dev = iv_ptr.device
+    # an empty run list still needs valid pointers
+    st = starts if starts.numel() else torch.zeros(1, dtype=torch.int16, device=dev)
+    ln = lens if lens.numel() else torch.zeros(1, dtype=torch.int16, device=dev)
+    row_ptr = torch.empty(H * nq + 1, dtype=torch.int32, device=dev)
+    _check("calib_intervals_to_csr", lib().calib_intervals_to_csr(
+        _ptr(iv_ptr), _ptr(st), _ptr(ln), H, nq, _ptr(row_ptr), None, _stream()))
+    nnz = int(row_ptr[-1].item())
+    col_idx = torch.empty(max(1, nnz), dtype=torch.int16, device=dev)
+    _check("calib_intervals_to_csr", lib().calib_intervals_to_csr(
+        _ptr(iv_ptr), _ptr(st), _ptr(ln), H, nq, _ptr(row_ptr), _ptr(col_idx), _stream()))
+    return row_ptr, col_idx[:nnz]
 
 
 def build_schedule(row_ptr: torch.Tensor, H: int, nq: int) -> torch.Tensor:

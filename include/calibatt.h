@@ -128,6 +128,26 @@ calib_status calib_aggregate_masks(const int32_t* counts, int H, int nq, int nk,
 calib_status calib_mask_to_csr(const uint8_t* mask, int H, int nq, int nk,
                                int32_t* row_ptr_out, int16_t* col_idx_out, void* stream);
 
+/* Interval form of a skip list ([zh] §2.2B and [fr] §2.C describe the per-query-block
+ * list as the block intervals to compute): every row's ascending kept key blocks grouped
+ * into maximal runs of consecutive indices.
+ *   row_ptr, col_idx : a CSR skip list (calib_mask_to_csr), col_idx ascending per row.
+ *   iv_ptr_out       : int32 [H*nq + 1], runs of row r at [iv_ptr[r], iv_ptr[r+1]).
+ *   iv_start_out     : int16, first key block of each run; iv_len_out: int16, its length.
+ *                      Capacity: the number of kept blocks (row_ptr[H*nq]) always suffices.
+ * Exact integer work; rows in order, runs in ascending order within a row. */
+calib_status calib_csr_to_intervals(const int32_t* row_ptr, const int16_t* col_idx, int H, int nq,
+                                    int32_t* iv_ptr_out, int16_t* iv_start_out,
+                                    int16_t* iv_len_out, void* stream);
+
+/* Inverse of calib_csr_to_intervals: expands runs back into the CSR skip list the
+ * attention kernel walks.  row_ptr_out int32 [H*nq + 1]; col_idx_out int16 with capacity
+ * for every kept block (the sum of all run lengths), or NULL: then only row_ptr_out is
+ * written, and its last entry sizes the list for a second call. */
+calib_status calib_intervals_to_csr(const int32_t* iv_ptr, const int16_t* iv_start,
+                                    const int16_t* iv_len, int H, int nq,
+                                    int32_t* row_ptr_out, int16_t* col_idx_out, void* stream);
+
 /* Processing order ([AdaSpa] §2 balances kernel load across heads of different
  * sparsity): work_out int32 [H*nq] = every row h << 16 | i, heads ascending and, within
  * a head, kept count descending (longest first), ties by i ascending.  Head-major order

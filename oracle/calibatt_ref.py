@@ -216,6 +216,40 @@ def mask_to_csr(mask: np.ndarray):
     return row_ptr.astype(np.int32), col_idx.astype(np.int16)
 
 
+def csr_to_intervals(row_ptr: np.ndarray, col_idx: np.ndarray):
+    """Interval form of a skip list: per row, the maximal runs of consecutive kept key
+    blocks as (start, length), in ascending order.
+
+    The pages describe the per-query-block list as the block intervals to compute ([zh]
+    §2.2B, [fr] §2.C).  Layout: iv_ptr int32 [rows + 1], starts int16, lengths int16."""
+    rp = np.asarray(row_ptr, np.int64)
+    ci = np.asarray(col_idx, np.int64)
+    iv_ptr, starts, lens = [0], [], []
+    for r in range(len(rp) - 1):
+        cols = ci[rp[r]:rp[r + 1]]
+        p = 0
+        while p < len(cols):
+            q = p + 1
+            while q < len(cols) and cols[q] == cols[q - 1] + 1:
+                q += 1
+            starts.append(cols[p])
+            lens.append(q - p)
+            p = q
+        iv_ptr.append(len(starts))
+    return (np.array(iv_ptr, np.int32), np.array(starts, np.int16), np.array(lens, np.int16))
+
+
+def intervals_to_csr(iv_ptr: np.ndarray, starts: np.ndarray, lens: np.ndarray):
+    """Inverse of csr_to_intervals: every run expanded into its block indices."""
+    ip = np.asarray(iv_ptr, np.int64)
+    row_ptr, cols = [0], []
+    for r in range(len(ip) - 1):
+        for k in range(ip[r], ip[r + 1]):
+            cols.extend(range(int(starts[k]), int(starts[k]) + int(lens[k])))
+        row_ptr.append(len(cols))
+    return np.array(row_ptr, np.int32), np.array(cols, np.int16)
+
+
 def build_schedule(row_ptr: np.ndarray, H: int, nq: int) -> np.ndarray:
     """Work list for load balancing by kept-block count: heads in ascending order and,
     within a head, query blocks by kept count descending (ties by query block

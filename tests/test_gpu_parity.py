@@ -166,6 +166,44 @@ def test_csr_and_schedule_bit_exact(H, nq, nk):
     np.testing.assert_array_equal(w, oracle.build_schedule(rp_ref, H, nq))
 
 
+@pytest.mark.parametrize("H,nq,nk,p", [(3, 40, 70, 0.1), (2, 33, 257, 0.5), (4, 17, 1000, 0.95)])
+def test_intervals_bit_exact_and_round_trip(H, nq, nk, p):
+    rng = np.random.default_rng(nq * 7 + nk)
+    m = _rand_mask(rng, H, nq, nk, p=p, diag=False)
+    m[0, 0] = 0
+    m[-1, -1] = 1
+    rp, ci = oracle.mask_to_csr(m)
+    ip_ref, st_ref, ln_ref = oracle.csr_to_intervals(rp, ci)
+    rp_t = torch.from_numpy(rp).cuda()
+    ci_t = torch.from_numpy(ci).cuda()
+    ip, st, ln = ops.csr_to_intervals(rp_t, ci_t, H, nq)
+    np.testing.assert_array_equal(ip.cpu().numpy(), ip_ref)
+    np.testing.assert_array_equal(st.cpu().numpy(), st_ref)
+    np.testing.assert_array_equal(ln.cpu().numpy(), ln_ref)
+    rp2, ci2 = ops.intervals_to_csr(ip, st, ln, H, nq)
+    np.testing.assert_array_equal(rp2.cpu().numpy(), rp)
+    np.testing.assert_array_equal(ci2.cpu().numpy(), ci)
+
+
+def test_intervals_generator_masks_and_empty_list():
+    wl = synth.WORKLOADS["wan13b"]
+    m = synth.make_head_masks(wl)[:3]
+    H, nq, _ = m.shape
+    bl = ops.BlockList.from_mask(torch.from_numpy(m).cuda(), wl.shape.block)
+    ip, st, ln = ops.csr_to_intervals(bl.row_ptr, bl.col_idx, H, nq)
+    ip_ref, st_ref, ln_ref = oracle.csr_to_intervals(*oracle.mask_to_csr(m))
+    np.testing.assert_array_equal(ip.cpu().numpy(), ip_ref)
+    np.testing.assert_array_equal(st.cpu().numpy(), st_ref)
+    np.testing.assert_array_equal(ln.cpu().numpy(), ln_ref)
+    # a list with no kept block at all
+    z = np.zeros((2, 5, 9), np.uint8)
+    rp, ci = ops.mask_to_csr(torch.from_numpy(z).cuda())
+    ip, st, ln = ops.csr_to_intervals(rp, ci, 2, 5)
+    assert int(ip[-1]) == 0 and st.numel() == 0
+    rp2, ci2 = ops.intervals_to_csr(ip, st, ln, 2, 5)
+    assert rp2.cpu().numpy().tolist() == [0] * 11 and ci2.numel() == 0
+
+
 @pytest.mark.parametrize("geom", [(4, 8, 16, 0, 2), (21, 45, 80, 0, 4), (28, 30, 53, 256, 4), (3, 7, 5, 9, 3),
                                   (2, 5, 3, 0, 1)])
 def test_anchor_rows_exact(geom):
@@ -210,6 +248,22 @@ def test_energy_cached_lse_and_accumulate(tiny_inputs):
     acc = ops.block_energy(q.cuda(), k.cuda(), B, accumulate=True)
     acc = ops.block_energy(q.cuda(), k.cuda(), B, out=acc, accumulate=True)
     check_energy(acc, 2 * ref, wl.shape.N, B)
+
+
+@pytest.mark.parametrize("geom", [(2, 64, 4, 8, 16, 64), (2, 128, 6, 10, 23, 128)])
+def test_energy_from_attention_lse(geom):
+    """LSE reuse (the AdaSpa-style step): a dense forward emits the row LSE, and the energy
+    pass takes it and runs a single pass.  The result must match the oracle's energies
+    (exact fp64 LSE), which two-pass energies do as well."""
+    H, D, F, Hl, Wl, B = geom
+    wl = _shape(H, D, F, Hl, Wl, B)
+    q, k, v = _inputs(wl, seed=41)
+    N = wl.shape.N
+    nb = -(-N // B)
+    _, lse = ops.sparse_attn_fwd(q, k, v, _blist(np.ones((H, nb, nb), np.uint8), B), return_lse=True)
+    ref = oracle.block_energy(to64(q), to64(k), 1.0 / math.sqrt(D), B)
+    got = ops.block_energy(q, k, B, lse=lse)
+    check_energy(got, ref, N, B)
 
 
 def test_energy_anchor_rows(tiny_inputs):
