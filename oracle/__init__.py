@@ -24,6 +24,6 @@ here is "parity unpinned".
 from .calibatt_ref import (  # noqa: F401
     logits, row_lse, block_energy, energy_mean, quantize_row, select_row, select_mask,
     aggregate_masks, mask_to_csr, csr_to_intervals, intervals_to_csr, build_schedule, anchor_rows,
-    anchor_index_of_token,
+    anchor_index_of_token, anchor_token, repeat_similarity, repeat_flags,
     sparse_attention, sparse_attention_repeat, ceil_log2,
 )

@@ -302,6 +302,53 @@ def anchor_index_of_token(t: int, F: int, Hl: int, Wl: int, n_text: int, stride:
     return (f * Ar + y // stride) * Wl + x
 
 
+def anchor_token(t: int, F: int, Hl: int, Wl: int, stride: int) -> int:
+    """Token whose attention row video token t = (f, y, x) takes at stride s: the anchor
+    (f, floor(y/s)*s, x).  Text tokens (t >= F*Hl*Wl) are their own anchor."""
+    nv = F * Hl * Wl
+    if t >= nv:
+        return t
+    x = t % Wl
+    y = (t // Wl) % Hl
+    f = t // (Wl * Hl)
+    return (f * Hl + (y // stride) * stride) * Wl + x
+
+
+def repeat_similarity(q: np.ndarray, k: np.ndarray, scale: float, members, F: int, Hl: int, Wl: int,
+                      stride: int) -> np.ndarray:
+    """cos(P[a(b)], P[b]) for every sampled token b and head h: [H, n].
+
+    [zh] §2.2A: the cosine similarity between the attention vectors of different spatial
+    rows of one frame is measured; a head whose similarity exceeds gamma is marked spatially
+    repetitive ([fr] §2.B.3 likewise).  Reading: a token's attention vector is its
+    post-softmax row P over all keys, and each sampled token b = (f, y, x) is compared with
+    the anchor a(b) = (f, floor(y/s)*s, x) whose output it would receive."""
+    H = q.shape[0]
+    members = [int(b) for b in members]
+    anchors = [anchor_token(b, F, Hl, Wl, stride) for b in members]
+    out = np.empty((H, len(members)), np.float64)
+    for h in range(H):
+        rows = sorted(set(members) | set(anchors))
+        idx = {r: n for n, r in enumerate(rows)}
+        S = logits(q[h][rows], k[h], scale)
+        P = np.exp(S - S.max(axis=1, keepdims=True))
+        P /= P.sum(axis=1, keepdims=True)
+        for i, (a, b) in enumerate(zip(anchors, members)):
+            pa, pb = P[idx[a]], P[idx[b]]
+            out[h, i] = float(pa @ pb) / np.sqrt(float(pa @ pa) * float(pb @ pb))
+    return out
+
+
+def repeat_flags(sim: np.ndarray, members, F: int, Hl: int, Wl: int, stride: int, gamma: float):
+    """Per head: the mean similarity over the sampled tokens that are not their own anchor,
+    and the flag mean > gamma ("exceeds the threshold", [zh] §2.2A).  A head with no such
+    token is not flagged (mean 0)."""
+    use = np.array([anchor_token(int(b), F, Hl, Wl, stride) != int(b) for b in members], bool)
+    sim = np.asarray(sim, np.float64)
+    mean = sim[:, use].mean(axis=1) if use.any() else np.zeros(sim.shape[0])
+    return mean, mean > gamma
+
+
 # ---------------------------------------------------------------------------------
 # Block-sparse attention
 # ---------------------------------------------------------------------------------
