@@ -1,0 +1,149 @@
+"""The calibrated mask dictionary: one static block mask per (timestep t, layer l, head h).
+
+The method calibrates offline and keeps, per timestep, layer and head, a static block mask
+(plus the spatial-repetition flag of the head) that inference looks up instead of searching
+([zh] §2.2A-§2.2B, [de] §2A.5 and §2B, [fr] §2.B.3 and §2.C of the summaries of
+"Accelerating Text-to-Video Generation with Calibrated Sparse Attention").  Here one
+(t, l) slice covers all H heads:
+
+* on the device, a slice is kept in interval form (runs of consecutive kept key blocks per
+  row, calib_csr_to_intervals) and expanded on demand into the CSR skip list plus the
+  longest-first schedule the attention kernel walks (calib_intervals_to_csr,
+  calib_build_schedule);
+* on disk, the dictionary is one little-endian file:
+
+      b"CBSDICT1"
+      int32[8]  T, L, H, nq, nk, block, stride, n_slices
+      n_slices x {
+          int32[3]  t, l, n_runs
+          uint8[H]  repeat flag of every head, zero-padded to a multiple of 4 bytes
+          int32[H*nq + 1]  run offsets per row
+          int16[n_runs]    run starts
+          int16[n_runs]    run lengths, zero-padded to a multiple of 4 bytes
+      }
+
+Repeat heads use anchor-space query blocks: their rows past the anchor sequence are empty.
+Every conversion runs in the library's kernels; this module only moves buffers and bytes.
+"""
+from __future__ import annotations
+
+import struct
+from dataclasses import dataclass, field
+from typing import Dict, Optional, Sequence, Tuple
+
+import numpy as np
+import torch
+
+from . import ops
+
+MAGIC = b"CBSDICT1"
+
+
+@dataclass
+class _Slice:
+    iv_ptr: torch.Tensor          # int32 [H*nq + 1]
+    starts: torch.Tensor          # int16 [n_runs]
+    lens: torch.Tensor            # int16 [n_runs]
+    repeat: Tuple[bool, ...]      # [H]
+
+
+@dataclass
+class MaskDictionary:
+    T: int
+    L: int
+    H: int
+    nq: int
+    nk: int
+    block: int
+    stride: int = 1
+    slices: Dict[Tuple[int, int], _Slice] = field(default_factory=dict)
+    _lists: Dict[Tuple[int, int], ops.BlockList] = field(default_factory=dict, repr=False)
+
+    # ---- building ----------------------------------------------------------------
+    def put_mask(self, t: int, l: int, mask: torch.Tensor, repeat: Optional[Sequence[bool]] = None):
+        """Store the (t, l) slice from a uint8 [H, nq, nk] device mask (anchor-space rows for
+        repeat heads)."""
+        self._check_key(t, l)
+        if tuple(mask.shape) != (self.H, self.nq, self.nk):
+            raise ValueError(f"mask shape {tuple(mask.shape)} != {(self.H, self.nq, self.nk)}")
+        row_ptr, col_idx = ops.mask_to_csr(mask)
+        self.put_csr(t, l, row_ptr, col_idx, repeat)
+
+    def put_csr(self, t: int, l: int, row_ptr: torch.Tensor, col_idx: torch.Tensor,
+                repeat: Optional[Sequence[bool]] = None):
+        self._check_key(t, l)
+        iv_ptr, starts, lens = ops.csr_to_intervals(row_ptr, col_idx, self.H, self.nq)
+        rep = tuple(bool(x) for x in (repeat if repeat is not None else [False] * self.H))
+        if len(rep) != self.H:
+            raise ValueError("repeat needs one flag per head")
+        self.slices[(t, l)] = _Slice(iv_ptr, starts.clone(), lens.clone(), rep)
+        self._lists.pop((t, l), None)
+
+    # ---- lookup ------------------------------------------------------------------
+    def block_list(self, t: int, l: int) -> ops.BlockList:
+        """CSR skip list + schedule of slice (t, l), expanded on first use and cached."""
+        key = (t, l)
+        if key not in self._lists:
+            s = self.slices[key]
+            row_ptr, col_idx = ops.intervals_to_csr(s.iv_ptr, s.starts, s.lens, self.H, self.nq)
+            work = ops.build_schedule(row_ptr, self.H, self.nq)
+            self._lists[key] = ops.BlockList(self.H, self.nq, self.nk, self.block, row_ptr, col_idx, work)
+        return self._lists[key]
+
+    def repeat_heads(self, t: int, l: int) -> Tuple[bool, ...]:
+        return self.slices[(t, l)].repeat
+
+    def _check_key(self, t: int, l: int):
+        if not (0 <= t < self.T and 0 <= l < self.L):
+            raise KeyError(f"(t, l) = {(t, l)} outside T={self.T}, L={self.L}")
+
+    # ---- files -------------------------------------------------------------------
+    def to_bytes(self) -> bytes:
+        out = [MAGIC, struct.pack("<8i", self.T, self.L, self.H, self.nq, self.nk, self.block, self.stride,
+                                  len(self.slices))]
+        for (t, l) in sorted(self.slices):
+            s = self.slices[(t, l)]
+            n = s.starts.numel()
+            out.append(struct.pack("<3i", t, l, n))
+            rep = np.array(s.repeat, np.uint8).tobytes()
+            out.append(rep + b"\0" * (-len(rep) % 4))
+            out.append(s.iv_ptr.cpu().numpy().astype("<i4").tobytes())
+            runs = s.starts.cpu().numpy().astype("<i2").tobytes() + s.lens.cpu().numpy().astype("<i2").tobytes()
+            out.append(runs + b"\0" * (-len(runs) % 4))
+        return b"".join(out)
+
+    def save(self, path: str):
+        with open(path, "wb") as f:
+            f.write(self.to_bytes())
+
+    @classmethod
+    def from_bytes(cls, buf: bytes, device="cuda") -> "MaskDictionary":
+        if buf[:8] != MAGIC:
+            raise ValueError("not a calibrated mask dictionary (bad magic)")
+        T, L, H, nq, nk, block, stride, n_slices = struct.unpack_from("<8i", buf, 8)
+        d = cls(T, L, H, nq, nk, block, stride)
+        off = 40
+        for _ in range(n_slices):
+            t, l, n = struct.unpack_from("<3i", buf, off)
+            off += 12
+            rep = tuple(bool(x) for x in np.frombuffer(buf, np.uint8, H, off))
+            off += H + (-H % 4)
+            iv_ptr = np.frombuffer(buf, "<i4", H * nq + 1, off).astype(np.int32)
+            off += 4 * (H * nq + 1)
+            starts = np.frombuffer(buf, "<i2", n, off).astype(np.int16)
+            lens = np.frombuffer(buf, "<i2", n, off + 2 * n).astype(np.int16)
+            off += 4 * n + (-(4 * n) % 4)
+            if int(iv_ptr[-1]) != n:
+                raise ValueError(f"slice {(t, l)}: run offsets end at {int(iv_ptr[-1])}, expected {n}")
+            d._check_key(t, l)
+            d.slices[(t, l)] = _Slice(torch.from_numpy(iv_ptr.copy()).to(device),
+                                      torch.from_numpy(starts.copy()).to(device),
+                                      torch.from_numpy(lens.copy()).to(device), rep)
+        if off != len(buf):
+            raise ValueError(f"{len(buf) - off} trailing bytes")
+        return d
+
+    @classmethod
+    def load(cls, path: str, device="cuda") -> "MaskDictionary":
+        with open(path, "rb") as f:
+            return cls.from_bytes(f.read(), device)

@@ -1,0 +1,63 @@
+"""The mask dictionary's file format, round-tripped on the CPU with oracle-made slices
+(no kernel involved): every array, flag and header field survives, and damaged files are
+rejected."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from calibrated_block_sparse_calib_b200.dictionary import MaskDictionary, _Slice, MAGIC
+
+
+def _dict(seed=0):
+    rng = np.random.default_rng(seed)
+    T, L, H, nq, nk = 3, 2, 3, 7, 11
+    d = MaskDictionary(T, L, H, nq, nk, block=64, stride=4)
+    ref = {}
+    for t in range(T):
+        for l in range(L):
+            if (t, l) == (2, 1):
+                continue                                  # a missing slice stays missing
+            m = (rng.random((H, nq, nk)) < 0.1 + 0.3 * t).astype(np.uint8)
+            ip, st, ln = oracle.csr_to_intervals(*oracle.mask_to_csr(m))
+            rep = tuple(bool(x) for x in rng.random(H) < 0.5)
+            d.slices[(t, l)] = _Slice(torch.from_numpy(ip), torch.from_numpy(st), torch.from_numpy(ln), rep)
+            ref[(t, l)] = (m, ip, st, ln, rep)
+    return d, ref
+
+
+def test_round_trip_every_field():
+    d, ref = _dict()
+    buf = d.to_bytes()
+    assert buf[:8] == MAGIC
+    e = MaskDictionary.from_bytes(buf, device="cpu")
+    assert (e.T, e.L, e.H, e.nq, e.nk, e.block, e.stride) == (3, 2, 3, 7, 11, 64, 4)
+    assert set(e.slices) == set(ref)
+    for key, (m, ip, st, ln, rep) in ref.items():
+        s = e.slices[key]
+        np.testing.assert_array_equal(s.iv_ptr.numpy(), ip)
+        np.testing.assert_array_equal(s.starts.numpy(), st)
+        np.testing.assert_array_equal(s.lens.numpy(), ln)
+        assert s.repeat == rep
+        # the runs still describe the original mask
+        rp, ci = oracle.intervals_to_csr(s.iv_ptr.numpy(), s.starts.numpy(), s.lens.numpy())
+        np.testing.assert_array_equal((rp, ci)[0], oracle.mask_to_csr(m)[0])
+        np.testing.assert_array_equal(ci, oracle.mask_to_csr(m)[1])
+    assert e.to_bytes() == buf
+
+
+def test_damaged_files_are_rejected():
+    d, _ = _dict(1)
+    buf = d.to_bytes()
+    with pytest.raises(ValueError):
+        MaskDictionary.from_bytes(b"XXXXXXXX" + buf[8:], device="cpu")
+    with pytest.raises(ValueError):
+        MaskDictionary.from_bytes(buf + b"\0\0\0\0", device="cpu")
+    with pytest.raises(Exception):
+        MaskDictionary.from_bytes(buf[:-4], device="cpu")
+
+
+def test_keys_outside_the_grid_are_rejected():
+    d = MaskDictionary(2, 2, 1, 1, 1, 64)
+    with pytest.raises(KeyError):
+        d._check_key(2, 0)

@@ -524,3 +524,35 @@ def test_mochi1_text_tokens_sampled():
     qh, kh, vh = (to64(t[heads]) for t in (q, k, v))
     O_ref, _ = oracle.sparse_attention(qh, kh, vh, 1 / math.sqrt(s.D), s.block, mask[heads], q_blocks=blocks)
     check_attn(O[heads], O_ref, rows=rows)
+
+
+def test_mask_dictionary_build_save_load_attend(tmp_path):
+    """Dictionary of 2 timesteps x 2 layers built on the device (masks -> runs), saved,
+    loaded, expanded: skip lists bit-exact to the oracle's, and attention through the
+    loaded list bit-identical to attention through a list built from the mask."""
+    from calibrated_block_sparse_calib_b200.dictionary import MaskDictionary
+    wl = _shape(2, 64, 4, 8, 16, 64)
+    s = wl.shape
+    q, k, v = _inputs(wl, seed=5)
+    rng = np.random.default_rng(11)
+    nb = s.nblk
+    d = MaskDictionary(2, 2, s.H, nb, nb, s.block)
+    masks = {}
+    for t in range(2):
+        for l in range(2):
+            m = _rand_mask(rng, s.H, nb, nb, p=0.3 + 0.2 * t)
+            masks[(t, l)] = m
+            d.put_mask(t, l, torch.from_numpy(m).cuda(), repeat=[False, t == 1])
+    path = str(tmp_path / "masks.cbsd")
+    d.save(path)
+    e = MaskDictionary.load(path)
+    for (t, l), m in masks.items():
+        bl = e.block_list(t, l)
+        rp_ref, ci_ref = oracle.mask_to_csr(m)
+        np.testing.assert_array_equal(bl.row_ptr.cpu().numpy(), rp_ref)
+        np.testing.assert_array_equal(bl.col_idx.cpu().numpy(), ci_ref)
+        np.testing.assert_array_equal(bl.work.cpu().numpy(), oracle.build_schedule(rp_ref, s.H, nb))
+        assert e.repeat_heads(t, l) == (False, t == 1)
+        o1 = ops.sparse_attn_fwd(q, k, v, bl)
+        o2 = ops.sparse_attn_fwd(q, k, v, _blist(m, s.block))
+        assert torch.equal(o1, o2)
