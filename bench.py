@@ -444,6 +444,18 @@ def main():
                 "select_ms": ms_sel, "select_gbs": sel_bytes / (ms_sel * 1e-3) / 1e9,
                 "select_frac_hbm": sel_bytes / (ms_sel * 1e-3) / 1e9 / peaks["hbm_gbs"],
                 "tau": 0.95, "selected_density": float(msk.float().mean().item())}
+            # spatial-repetition detection: cosine of 1024 sampled tokens' attention rows
+            # against their stride-4 anchors, two passes over K, then the per-head decision
+            mem = torch.from_numpy(synth.sample_video_tokens(s, 1024, seed=1)).to(dev)
+            cos = ops.repeat_similarity(q, k, mem, s.F, s.Hl, s.Wl, 4)
+            ms_sim = _time_calls(lambda: ops.repeat_similarity(q, k, mem, s.F, s.Hl, s.Wl, 4), 3, 1, torch)
+            mean, flag = ops.repeat_flags(cos, mem, s.F, s.Hl, s.Wl, 4, 0.9)
+            rows_sim = 2 * 2 * mem.numel()          # anchor + sample rows, two passes
+            extras["calibration"]["repeat_detection"] = {
+                "samples": mem.numel(), "stride": 4, "gamma": 0.9, "ms": ms_sim,
+                "tflops_qk": 2.0 * rows_sim * N * D * H / (ms_sim * 1e-3) / 1e12,
+                "mean_similarity_min": float(mean.min().item()), "mean_similarity_max": float(mean.max().item()),
+                "heads_flagged": int(flag.sum().item())}
             # interval form of the default workload's skip list (mask storage)
             rows = H * s.nblk
             iv = ops.csr_to_intervals(bl.row_ptr, bl.col_idx, H, s.nblk)

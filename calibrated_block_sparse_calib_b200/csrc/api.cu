@@ -18,6 +18,7 @@
 #include "energy.cuh"
 #include "select.cuh"
 #include "intervals.cuh"
+#include "repeat_sim.cuh"
 
 namespace {
 
@@ -170,6 +171,18 @@ calib_status launch_energy(const CUtensorMap& tk, const calib::EnergyParams& p, 
     return launch_status();
 }
 
+// ---- spatial-repetition similarity -----------------------------------------------------
+template <int D, int BLK>
+calib_status launch_sim(const CUtensorMap& tk, const calib::SimParams& p, int grid, cudaStream_t st) {
+    constexpr int KST = 4;
+    using L = calib::SimSmem<D, BLK, KST>;
+    static_assert(L::BYTES <= 232448, "shared memory budget");
+    auto* fn = calib::repeat_sim_kernel<D, BLK, KST>;
+    if (calib_status s = ensure_smem(reinterpret_cast<const void*>(fn), L::BYTES)) return s;
+    fn<<<grid, calib::kEnergyThreads, L::BYTES, st>>>(tk, p);
+    return launch_status();
+}
+
 int rows_grid(long long rows) { return static_cast<int>((rows + 3) / 4); }   // 4 warps per block
 
 }  // namespace
@@ -296,6 +309,46 @@ calib_status calib_intervals_to_csr(const int32_t* iv_ptr, const int16_t* iv_sta
     if (col_idx_out)
         calib::iv_expand_kernel<<<rows_grid(rows), 128, 0, st>>>(iv_ptr, iv_start, iv_len, rows, row_ptr_out,
                                                                  col_idx_out);
+    return launch_status();
+}
+
+calib_status calib_repeat_similarity(const void* q, const void* k, const float* lse, int H, int N, int D, int block,
+                                     float scale, int F, int Hl, int Wl, int stride, const int32_t* members, int n,
+                                     float* cos_out, void* stream) {
+    if (!q || !k || !members || !cos_out || !aligned16(q) || !aligned16(k)) return CALIB_ERR_INVALID;
+    if ((reinterpret_cast<uintptr_t>(cos_out) & 3u) || (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
+        return CALIB_ERR_INVALID;
+    if (H < 1 || N < 1 || n < 1 || !(scale > 0.f) || !std::isfinite(scale)) return CALIB_ERR_INVALID;
+    if (F < 1 || Hl < 1 || Wl < 1 || stride < 1 || static_cast<long long>(F) * Hl * Wl > N) return CALIB_ERR_INVALID;
+    if (block != 64 && block != 128) return CALIB_ERR_INVALID;
+    if (D != 64 && D != 128) return CALIB_ERR_UNSUPPORTED;
+    const int tiles = cdiv(n, calib::kSimPairs);
+    if (static_cast<long long>(H) * tiles > (1ll << 31) - 1) return CALIB_ERR_INVALID;
+    if (calib_status s = check_device()) return s;
+    calib::SimParams p{};
+    p.q = static_cast<const __nv_bfloat16*>(q);
+    p.members = members;
+    p.lse_in = lse;
+    p.cos_out = cos_out;
+    p.H = H; p.N = N; p.n = n; p.tiles = tiles; p.nk = cdiv(N, block);
+    p.F = F; p.Hl = Hl; p.Wl = Wl; p.stride = stride;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.timeout_ns = kDefaultTimeoutNs;
+    CUtensorMap tk;
+    if (!make_tmap(&tk, k, D, N, H, block)) return CALIB_ERR_CUDA;
+    cudaStream_t st = as_stream(stream);
+    const int grid = H * tiles;
+    if (D == 128) return block == 128 ? launch_sim<128, 128>(tk, p, grid, st) : launch_sim<128, 64>(tk, p, grid, st);
+    return block == 128 ? launch_sim<64, 128>(tk, p, grid, st) : launch_sim<64, 64>(tk, p, grid, st);
+}
+
+calib_status calib_repeat_flags(const float* cos, const int32_t* members, int H, int n, int F, int Hl, int Wl,
+                                int stride, float gamma, float* mean_out, uint8_t* flag_out, void* stream) {
+    if (!cos || !members || !mean_out || !flag_out) return CALIB_ERR_INVALID;
+    if (H < 1 || n < 1 || F < 1 || Hl < 1 || Wl < 1 || stride < 1 || !std::isfinite(gamma)) return CALIB_ERR_INVALID;
+    if (calib_status s = check_device()) return s;
+    calib::repeat_flags_kernel<<<H, 256, 0, as_stream(stream)>>>(cos, members, n, F, Hl, Wl, stride, gamma, mean_out,
+                                                                  flag_out);
     return launch_status();
 }
 

@@ -45,6 +45,8 @@ _SIGS = {
     "calib_mask_to_csr": ([_P, _I, _I, _I, _P, _P, _P], ctypes.c_int),
     "calib_build_schedule": ([_P, _I, _I, _P, _P], ctypes.c_int),
     "calib_csr_to_intervals": ([_P, _P, _I, _I, _P, _P, _P, _P], ctypes.c_int),
+    "calib_repeat_similarity": ([_P, _P, _P, _I, _I, _I, _I, _F, _I, _I, _I, _I, _P, _I, _P, _P], ctypes.c_int),
+    "calib_repeat_flags": ([_P, _P, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P], ctypes.c_int),
     "calib_intervals_to_csr": ([_P, _P, _P, _I, _I, _P, _P, _P], ctypes.c_int),
     "calib_anchor_count": ([_I, _I, _I, _I, _I], ctypes.c_int64),
     "calib_anchor_rows": ([_I, _I, _I, _I, _I, _P, _P], ctypes.c_int),
@@ -215,6 +217,37 @@ def intervals_to_csr(iv_ptr: torch.Tensor, starts: torch.Tensor, lens: torch.Ten
     _check("calib_intervals_to_csr", lib().calib_intervals_to_csr(
         _ptr(iv_ptr), _ptr(st), _ptr(ln), H, nq, _ptr(row_ptr), _ptr(col_idx), _stream()))
     return row_ptr, col_idx[:nnz]
+
+
+def repeat_similarity(q: torch.Tensor, k: torch.Tensor, members: torch.Tensor, F: int, Hl: int, Wl: int,
+                      stride: int, block: int = 128, scale: Optional[float] = None,
+                      lse: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """fp32 [H, n]: cosine between the attention rows of each sampled token and its anchor."""
+    H, N, D = k.shape
+    _need(q, "q", torch.bfloat16, (H, N, D))
+    _need(k, "k", torch.bfloat16)
+    _need(members, "members", torch.int32)
+    if lse is not None:
+        _need(lse, "lse", torch.float32, (H, N))
+    n = members.numel()
+    out = torch.empty((H, n), dtype=torch.float32, device=q.device)
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    _check("calib_repeat_similarity", lib().calib_repeat_similarity(
+        _ptr(q), _ptr(k), _ptr(lse), H, N, D, block, scale, F, Hl, Wl, stride, _ptr(members), n, _ptr(out),
+        _stream()))
+    return out
+
+
+def repeat_flags(cos: torch.Tensor, members: torch.Tensor, F: int, Hl: int, Wl: int, stride: int, gamma: float):
+    """(mean fp32 [H], flag uint8 [H]): mean similarity over non-anchor samples, flag mean > gamma."""
+    _need(cos, "cos", torch.float32)
+    _need(members, "members", torch.int32)
+    H, n = cos.shape
+    mean = torch.empty(H, dtype=torch.float32, device=cos.device)
+    flag = torch.empty(H, dtype=torch.uint8, device=cos.device)
+    _check("calib_repeat_flags", lib().calib_repeat_flags(
+        _ptr(cos), _ptr(members), H, n, F, Hl, Wl, stride, float(gamma), _ptr(mean), _ptr(flag), _stream()))
+    return mean, flag
 
 
 def build_schedule(row_ptr: torch.Tensor, H: int, nq: int) -> torch.Tensor:

@@ -241,3 +241,9 @@ def anchor_block_count(shape: VideoShape, stride: int) -> int:
     F * ceil(Hl/stride) * Wl anchor tokens plus the text tokens, in blocks of B."""
     n_anchor = shape.F * (-(-shape.Hl // stride)) * shape.Wl + shape.n_text
     return (n_anchor + shape.block - 1) // shape.block
+
+
+def sample_video_tokens(shape: VideoShape, n: int, seed: int = 0) -> np.ndarray:
+    """n seeded video-token indices, uniform over the F*Hl*Wl video tokens (int32)."""
+    rng = np.random.default_rng(seed)
+    return rng.integers(0, shape.F * shape.Hl * shape.Wl, size=n).astype(np.int32)

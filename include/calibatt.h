@@ -148,6 +148,30 @@ calib_status calib_intervals_to_csr(const int32_t* iv_ptr, const int16_t* iv_sta
                                     const int16_t* iv_len, int H, int nq,
                                     int32_t* row_ptr_out, int16_t* col_idx_out, void* stream);
 
+/* Spatial-repetition detection, similarity step ([zh] §2.2A, [de] §2A.4, [fr] §2.B.3: the
+ * cosine similarity of attention vectors of different spatial rows of one frame):
+ *   cos_out[h, i] = cos(P_h[a(b_i)], P_h[b_i]) for every sampled token b_i, where P_h is
+ *   the post-softmax attention of head h over all N keys and a(b) = (f, floor(y/s)*s, x) is
+ *   the anchor of b = (f, y, x) at stride s (text tokens are their own anchor).
+ *   q, k     : bf16 [H, N, D], device, 16-byte aligned; token n = (f*Hl + y)*Wl + x for
+ *              the F*Hl*Wl video tokens, text tokens after them.
+ *   lse      : NULL (the row LSEs are computed: two passes over K) or fp32 [H, N].
+ *   members  : int32 [n] sampled token indices, shared by all heads (the caller draws them).
+ *   cos_out  : fp32 [H, n].
+ * P is never written to memory.  D in {64, 128}, block in {64, 128}. */
+calib_status calib_repeat_similarity(const void* q, const void* k, const float* lse,
+                                     int H, int N, int D, int block, float scale,
+                                     int F, int Hl, int Wl, int stride,
+                                     const int32_t* members, int n, float* cos_out, void* stream);
+
+/* Spatial-repetition detection, decision step: per head the mean of cos[h, i] over the
+ * samples that are not their own anchor, and flag = mean > gamma ("exceeds", [zh] §2.2A),
+ * taken in fp32.  A head with no such sample gets mean 0.  mean_out fp32 [H], flag_out
+ * uint8 [H]. */
+calib_status calib_repeat_flags(const float* cos, const int32_t* members, int H, int n,
+                                int F, int Hl, int Wl, int stride, float gamma,
+                                float* mean_out, uint8_t* flag_out, void* stream);
+
 /* Processing order ([AdaSpa] §2 balances kernel load across heads of different
  * sparsity): work_out int32 [H*nq] = every row h << 16 | i, heads ascending and, within
  * a head, kept count descending (longest first), ties by i ascending.  Head-major order

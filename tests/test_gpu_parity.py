@@ -556,3 +556,68 @@ def test_mask_dictionary_build_save_load_attend(tmp_path):
         o1 = ops.sparse_attn_fwd(q, k, v, bl)
         o2 = ops.sparse_attn_fwd(q, k, v, _blist(m, s.block))
         assert torch.equal(o1, o2)
+
+
+# ------------------------------------------------------------------------------------
+# spatial-repetition detection
+# ------------------------------------------------------------------------------------
+# Cosines are ratios of fp32 sums of N products of fp32 P values (ex2.approx, ~2^-22
+# relative) accumulated in 2 x 32 chains per half-row: worst-case relative rounding of a
+# sum ~ (N / 64) * 2^-24 per chain, i.e. ~1e-4 at N = 32K; held to 5e-4 absolute on cos.
+COS_ABS = 5e-4
+
+
+def _members(rng, shape, n):
+    return rng.integers(0, shape.F * shape.Hl * shape.Wl, size=n).astype(np.int32)
+
+
+@pytest.mark.parametrize("with_lse", [False, True])
+def test_repeat_similarity_tiny(tiny_inputs, with_lse):
+    wl, qkv = tiny_inputs
+    s = wl.shape
+    q, k, _ = (t.cuda() for t in qkv[0])
+    rng = np.random.default_rng(3)
+    mem = _members(rng, s, 150)
+    scale = 1.0 / math.sqrt(s.D)
+    ref = oracle.repeat_similarity(to64(q), to64(k), scale, mem, s.F, s.Hl, s.Wl, 2)
+    lse = None
+    if with_lse:
+        lse = torch.from_numpy(oracle.row_lse(to64(q), to64(k), scale).astype(np.float32)).cuda()
+    got = ops.repeat_similarity(q, k, torch.from_numpy(mem).cuda(), s.F, s.Hl, s.Wl, 2, block=s.block, lse=lse)
+    np.testing.assert_allclose(to64(got), ref, atol=COS_ABS, rtol=0)
+    mean_ref, flag_ref = oracle.repeat_flags(ref, mem, s.F, s.Hl, s.Wl, 2, 0.5)
+    mean, flag = ops.repeat_flags(got, torch.from_numpy(mem).cuda(), s.F, s.Hl, s.Wl, 2, 0.5)
+    np.testing.assert_allclose(to64(mean), mean_ref, atol=COS_ABS)
+    decisive = np.abs(mean_ref - 0.5) > COS_ABS
+    np.testing.assert_array_equal(flag.cpu().numpy().astype(bool)[decisive], flag_ref[decisive])
+
+
+def test_repeat_similarity_repeating_head_is_flagged():
+    """Head 1's member queries copy their anchors' queries: every cosine is 1 and the head is
+    flagged; head 0 (independent rows) is compared with the oracle."""
+    wl = _shape(2, 128, 3, 12, 20, 128)
+    s = wl.shape
+    q, k, _ = synth.make_qkv(wl, seed=9)
+    q = q.clone()
+    for t in range(s.F * s.Hl * s.Wl):
+        q[1, t] = q[1, oracle.anchor_token(t, s.F, s.Hl, s.Wl, 3)]
+    q, k = q.cuda(), k.cuda()
+    rng = np.random.default_rng(4)
+    mem = _members(rng, s, 200)
+    got = ops.repeat_similarity(q, k, torch.from_numpy(mem).cuda(), s.F, s.Hl, s.Wl, 3)
+    ref = oracle.repeat_similarity(to64(q), to64(k), 1.0 / math.sqrt(s.D), mem, s.F, s.Hl, s.Wl, 3)
+    np.testing.assert_allclose(to64(got), ref, atol=COS_ABS, rtol=0)
+    assert np.all(np.abs(to64(got)[1] - 1.0) < COS_ABS)
+    mean, flag = ops.repeat_flags(got, torch.from_numpy(mem).cuda(), s.F, s.Hl, s.Wl, 3, 0.99)
+    assert flag[1].item() == 1
+
+
+def test_repeat_similarity_wan13b_shape_sampled():
+    wl = synth.WORKLOADS["wan13b"]
+    s = wl.shape
+    q, k, _ = synth.make_qkv(wl, device="cuda", heads=2)
+    rng = np.random.default_rng(5)
+    mem = _members(rng, s, 96)
+    got = ops.repeat_similarity(q, k, torch.from_numpy(mem).cuda(), s.F, s.Hl, s.Wl, 4)
+    ref = oracle.repeat_similarity(to64(q), to64(k), 1.0 / math.sqrt(s.D), mem, s.F, s.Hl, s.Wl, 4)
+    np.testing.assert_allclose(to64(got), ref, atol=COS_ABS, rtol=0)
