@@ -265,6 +265,31 @@ def run_calibration_sweep(dev, torch, ops, synth):
         for tau in taus:
             dens["energy_sum"][str(tau)].append(float(ops.select_mask(Esum, tau, out=msk).float().mean().item()))
         del qk
+    # the dictionary of the sweep: one slice per timestep with a stricter tau early on
+    # (tau(t) = 0.99, 0.95, 0.9 over the three thirds of the schedule), repetition
+    # detection at gamma = 0.9 and stride 4, built by the calibration driver, saved, reloaded
+    from calibrated_block_sparse_calib_b200.calibrate import calibrate_slice
+    from calibrated_block_sparse_calib_b200.dictionary import MaskDictionary
+    import tempfile
+    dct = MaskDictionary(T, 1, H, nb, nb, B, stride=4)
+    members = torch.from_numpy(synth.sample_video_tokens(s, 512, seed=3)).to(dev)
+    t_d = time.perf_counter()
+    flags = []
+    for t in range(T):
+        tau_t = 0.99 if t < T // 3 else (0.95 if t < 2 * T // 3 else 0.9)
+        qk = [synth.make_qkv(wl, input_idx=d, device=dev, pos_scale=1.0 + 0.125 * t)[:2] for d in range(n_in)]
+        mask_t, rep_t, _ = calibrate_slice(qk, s.F, s.Hl, s.Wl, 0, B, tau_t, (1, 2), "vote", 0.9, 4, members)
+        dct.put_mask(t, 0, mask_t, rep_t)
+        flags.append(sum(rep_t))
+        del qk
+    torch.cuda.synchronize()
+    build_s = time.perf_counter() - t_d
+    with tempfile.TemporaryDirectory() as td:
+        path = os.path.join(td, "sweep.cbsd")
+        dct.save(path)
+        file_bytes = os.path.getsize(path)
+        back = MaskDictionary.load(path)
+        same = all(torch.equal(back.block_list(t, 0).col_idx, dct.block_list(t, 0).col_idx) for t in range(T))
     ops.device_check()
     em = statistics.median(e_ms)
     sm_ = statistics.median(sel_ms)
@@ -278,7 +303,12 @@ def run_calibration_sweep(dev, torch, ops, synth):
         "energy_tflops_qk": 2 * 2.0 * N * N * s.D * H / (em * 1e-3) / 1e12,
         "energy_accumulate_ms_median": statistics.median(a_ms),
         "select_ms_median": sm_, "select_gbs": sel_bytes / (sm_ * 1e-3) / 1e9,
-        "kept_density": dens, "wall_s": time.perf_counter() - t_start}), flush=True)
+        "kept_density": dens,
+        "dictionary": {"slices": T, "tau_schedule": [0.99 if t < T // 3 else (0.95 if t < 2 * T // 3 else 0.9)
+                                                     for t in range(T)],
+                       "repeat_heads_per_timestep": flags, "build_s": build_s, "file_bytes": file_bytes,
+                       "reload_identical": bool(same)},
+        "wall_s": time.perf_counter() - t_start}), flush=True)
 
 
 def main():

@@ -621,3 +621,50 @@ def test_repeat_similarity_wan13b_shape_sampled():
     got = ops.repeat_similarity(q, k, torch.from_numpy(mem).cuda(), s.F, s.Hl, s.Wl, 4)
     ref = oracle.repeat_similarity(to64(q), to64(k), 1.0 / math.sqrt(s.D), mem, s.F, s.Hl, s.Wl, 4)
     np.testing.assert_allclose(to64(got), ref, atol=COS_ABS, rtol=0)
+
+
+def test_calibrate_slice_with_repeat_head_bit_exact_from_gpu_energies():
+    """The calibration driver end to end on 3 inputs: head 1 (member queries copy their
+    anchors) is flagged and gets an anchor-space mask, head 0 a full-space one.  Replayed
+    with the oracle's selection, vote and repetition decision on the same GPU energies and
+    cosines, the slice mask is bit-exact."""
+    from calibrated_block_sparse_calib_b200.calibrate import calibrate_slice
+    wl = _shape(2, 64, 4, 8, 16, 64)
+    s = wl.shape
+    B, stride, tau, rho, gamma = s.block, 2, 0.9, (1, 2), 0.99
+    inputs = []
+    for d in range(3):
+        q, k, _ = synth.make_qkv(wl, seed=100 + d)
+        q = q.clone()
+        for t in range(s.N):
+            q[1, t] = q[1, oracle.anchor_token(t, s.F, s.Hl, s.Wl, stride)]
+        inputs.append((q.cuda(), k.cuda()))
+    members = torch.from_numpy(synth.sample_video_tokens(s, 120, seed=2)).cuda()
+    mask, repeat, det = calibrate_slice(inputs, s.F, s.Hl, s.Wl, 0, B, tau, rho, "vote", gamma, stride, members)
+    assert repeat == [False, True]
+    # replay with the oracle on the GPU's energies (bit-exact selection needs identical energies)
+    mem = members.cpu().numpy()
+    cos = np.concatenate([to64(ops.repeat_similarity(q, k, members, s.F, s.Hl, s.Wl, stride, B))
+                          for q, k in inputs], axis=1)
+    mean_ref, flag_ref = oracle.repeat_flags(cos, np.tile(mem, 3), s.F, s.Hl, s.Wl, stride, gamma)
+    assert flag_ref.tolist() == [False, True]
+    rows = ops.anchor_rows(s.F, s.Hl, s.Wl, 0, stride)
+    nb, nqa = s.nblk, -(-rows.numel() // B)
+    cnt_full = np.zeros((2, nb, nb), np.int64)
+    cnt_anch = np.zeros((2, nqa, nb), np.int64)
+    for q, k in inputs:
+        cnt_full += oracle.select_mask(ops.block_energy(q, k, B).cpu().numpy(), tau)
+        cnt_anch += oracle.select_mask(ops.block_energy(q, k, B, q_rows=rows).cpu().numpy(), tau)
+    ref = oracle.aggregate_masks(cnt_full, 3, *rho)
+    ref_a = oracle.aggregate_masks(cnt_anch, 3, *rho)
+    ref[1] = 0
+    ref[1, :nqa] = ref_a[1]
+    np.testing.assert_array_equal(mask.cpu().numpy(), ref)
+    # the slice's masks drive the repeat-mode attention as they are
+    bl = _blist(mask.cpu().numpy(), B)
+    q, k = inputs[0]
+    v = synth.make_qkv(wl, seed=100)[2].cuda()
+    O = ops.sparse_attn_fwd_repeat(q, k, v, bl, repeat, s.F, s.Hl, s.Wl, 0, stride)
+    O_ref, _ = oracle.sparse_attention_repeat(to64(q), to64(k), to64(v), 1.0 / math.sqrt(s.D), B,
+                                              mask.cpu().numpy(), repeat, s.F, s.Hl, s.Wl, 0, stride)
+    check_attn(O, O_ref)
