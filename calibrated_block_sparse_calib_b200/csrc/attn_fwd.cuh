@@ -157,6 +157,45 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     const int nkept = p.row_ptr[lrow + 1] - kbeg;
 
     // ---- setup ------------------------------------------------------------------
+    // The first softmax warps fetch their Q rows into registers now, so that the global
+    // load latency overlaps the setup (they store the rows into tensor memory after it).
+    constexpr int QW = D / 2;                          // 32-bit words of one Q row
+    uint32_t qrow[QW];
+    const bool q_loader = warp >= 2 && warp < 6 && nkept > 0;
+    if (q_loader) {
+        const int r = static_cast<int>((warp & 3) * 32 + lane);
+        const int a = i * BLK + r;
+        // rows past the block or the sequence are zero
+        const uint4* src = (r < BLK && a < Nq)
+                               ? reinterpret_cast<const uint4*>(
+                                     p.q + (static_cast<size_t>(h) * p.N + (rep ? anchor_token(p, a) : a)) * D)
+                               : nullptr;
+#pragma unroll
+        for (int v = 0; v < QW / 4; ++v) {
+            const uint4 x = src ? __ldg(src + v) : make_uint4(0, 0, 0, 0);
+            qrow[4 * v] = x.x;
+            qrow[4 * v + 1] = x.y;
+            qrow[4 * v + 2] = x.z;
+            qrow[4 * v + 3] = x.w;
+        }
+    }
+    if (warp == 0) {
+        // walk the list from the diagonal block: the first kept key block at or after the
+        // key block holding the query block's first token (the list is ascending, so one
+        // ballot over 32 entries at a time finds it)
+        const int tok = rep ? anchor_token(p, min(i * BLK, Nq - 1)) : i * BLK;
+        const int jd = tok / BLK;
+        int t0 = 0;
+        for (int b0 = 0; b0 < nkept; b0 += 32) {
+            const int x = b0 + static_cast<int>(lane);
+            const uint32_t ge = __ballot_sync(0xffffffffu, x < nkept && p.col_idx[kbeg + x] >= jd);
+            if (ge) {
+                t0 = b0 + __ffs(ge) - 1;
+                break;
+            }
+        }
+        if (lane == 0) *t0_slot = t0;
+    }
     if (threadIdx.x == 0) {
         mbar_init(bar(L::B_Q), 128u);
         for (int s = 0; s < KST; ++s) { mbar_init(bar(L::B_KF + s), 1); mbar_init(bar(L::B_KE + s), 1); }
@@ -167,13 +206,6 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         mbar_init(bar(L::B_O), 1);
         mbar_init(bar(L::B_DRAIN), 1);
         *abort_flag = 0;
-        // walk the list from the diagonal block: first kept key block at or after the
-        // key block holding the query block's first token
-        const int tok = rep ? anchor_token(p, min(i * BLK, Nq - 1)) : i * BLK;
-        const int jd = tok / BLK;
-        int t0 = 0;
-        while (t0 < nkept && p.col_idx[kbeg + t0] < jd) ++t0;
-        *t0_slot = t0 < nkept ? t0 : 0;
         fence_barrier_init();
     }
     if (warp == 0 && lane == 0) {
@@ -312,27 +344,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         const int r = static_cast<int>(q4 * 32 + lane);   // tile row == TMEM lane
         const uint32_t lane_base = (q4 * 32) << 16;
         const uint32_t o_col = kTmemO + hf * D;            // this half's accumulator O_h
-        if (nkept > 0 && hf == 0) {
+        if (q_loader) {
             // Q row -> tensor memory: the bf16 pairs of the row in memory order are the
-            // packed TS operand.  Rows past the block or the sequence are zero.
-            const int a = i * BLK + r;
-            const uint4* src = (r < BLK && a < Nq)
-                                   ? reinterpret_cast<const uint4*>(
-                                         p.q + (static_cast<size_t>(h) * p.N + (rep ? anchor_token(p, a) : a)) * D)
-                                   : nullptr;
-            uint32_t w[32];
+            // packed TS operand
 #pragma unroll
-            for (int c = 0; c < D / 64; ++c) {
-#pragma unroll
-                for (int v = 0; v < 8; ++v) {
-                    const uint4 x = src ? __ldg(src + c * 8 + v) : make_uint4(0, 0, 0, 0);
-                    w[4 * v] = x.x;
-                    w[4 * v + 1] = x.y;
-                    w[4 * v + 2] = x.z;
-                    w[4 * v + 3] = x.w;
-                }
-                tmem_st32(tmem + lane_base + kTmemQ + c * 32, w);
-            }
+            for (int c = 0; c < D / 64; ++c)
+                tmem_st32(tmem + lane_base + kTmemQ + c * 32, *reinterpret_cast<const uint32_t(*)[32]>(qrow + c * 32));
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(bar(L::B_Q));
