@@ -668,3 +668,85 @@ def test_calibrate_slice_with_repeat_head_bit_exact_from_gpu_energies():
     O_ref, _ = oracle.sparse_attention_repeat(to64(q), to64(k), to64(v), 1.0 / math.sqrt(s.D), B,
                                               mask.cpu().numpy(), repeat, s.F, s.Hl, s.Wl, 0, stride)
     check_attn(O, O_ref)
+
+
+# ------------------------------------------------------------------------------------
+# fixtures under tests/golden/: hand-worked cases and the Tiny workload's stored oracle
+# results (no oracle call at test time)
+# ------------------------------------------------------------------------------------
+
+from golden_data import hand_worked, tiny_calibration  # noqa: E402
+
+_HW = hand_worked()
+
+
+@pytest.mark.parametrize("case", _HW["select"], ids=lambda c: f"line{c['line']}")
+def test_hand_worked_select_kernel(case):
+    nk, i = len(case["e"]), case["diag"]
+    E = np.zeros((1, i + 1, nk), np.float32)
+    E[0, i] = case["e"]
+    fk = None
+    if case["forced"] is not None:
+        f = np.zeros((1, i + 1, nk), np.uint8)
+        f[0, i] = case["forced"]
+        fk = torch.from_numpy(f).cuda()
+    m = ops.select_mask(torch.from_numpy(E).cuda(), case["tau"], force_keep=fk).cpu().numpy()
+    np.testing.assert_array_equal(m[0, i], case["keep"])
+
+
+@pytest.mark.parametrize("case", _HW["vote"], ids=lambda c: f"line{c['line']}")
+def test_hand_worked_vote_kernel(case):
+    c = torch.from_numpy(case["counts"].astype(np.int32)[None, None]).cuda()
+    np.testing.assert_array_equal(ops.aggregate_masks(c, case["n"], case["rho"]).cpu().numpy()[0, 0], case["keep"])
+
+
+@pytest.mark.parametrize("case", _HW["runs"], ids=lambda c: f"line{c['line']}")
+def test_hand_worked_runs_kernel(case):
+    rp, ci = ops.mask_to_csr(torch.from_numpy(case["row"][None, None]).cuda())
+    ip, st, ln = ops.csr_to_intervals(rp, ci, 1, 1)
+    assert st.cpu().tolist() == case["starts"] and ln.cpu().tolist() == case["lens"]
+    assert ip.cpu().tolist() == [0, len(case["starts"])]
+
+
+@pytest.mark.parametrize("case", _HW["anchors"], ids=lambda c: f"line{c['line']}")
+def test_hand_worked_anchor_rows_kernel(case):
+    rows = ops.anchor_rows(case["F"], case["Hl"], case["Wl"], case["text"], case["stride"])
+    assert rows.cpu().tolist() == case["rows"]
+
+
+def test_tiny_golden_pipeline():
+    """The Tiny workload through the kernels against the stored oracle results: energies
+    in both query spaces within 1e-4 relative; selection from the stored energies, the
+    vote, the skip list and the work order bit-exact; sampled attention rows (repeat head
+    included) within the attention bar."""
+    g = tiny_calibration()
+    w = g["workload"]
+    wl = synth.WORKLOADS["tiny"]
+    B = w["block"]
+    qkv = [synth.make_qkv(wl, input_idx=d) for d in range(w["n_inputs"])]
+    rows_a = ops.anchor_rows(w["F"], w["Hl"], w["Wl"], w["n_text"], w["stride"])
+    for name, sp in g["spaces"].items():
+        q_rows = rows_a if name == "anchor" else None
+        Nq = w["n_anchor"] if name == "anchor" else w["N"]
+        counts = torch.zeros(tuple(sp["shape"]), dtype=torch.int32, device="cuda")
+        for (q, k, _), e_ref, m_ref in zip(qkv, sp["energy_f32"], sp["mask_arrays"]):
+            e_gpu = ops.block_energy(q.cuda(), k.cuda(), B, q_rows=q_rows)
+            check_energy(e_gpu, e_ref.astype(np.float64), Nq, B)
+            m = ops.select_mask(torch.from_numpy(e_ref).cuda(), w["tau"], count_accum=counts)
+            np.testing.assert_array_equal(m.cpu().numpy(), m_ref)
+        np.testing.assert_array_equal(counts.cpu().numpy(), sp["counts_array"])
+        vote = ops.aggregate_masks(counts, w["n_inputs"], w["rho"]).cpu().numpy()
+        np.testing.assert_array_equal(vote, sp["vote_array"])
+    sl = g["slice"]
+    bl = _blist(sl["mask_array"], B)
+    nnz = sl["row_ptr"][-1]
+    assert bl.row_ptr.cpu().tolist() == sl["row_ptr"]
+    assert bl.col_idx[:nnz].cpu().tolist() == sl["col_idx"]
+    assert bl.work.cpu().tolist() == sl["work"]
+    at = g["attention"]
+    q, k, v = (t.cuda() for t in qkv[at["input"]])
+    for out_dtype in (torch.float32, torch.bfloat16):
+        O, L = ops.sparse_attn_fwd_repeat(q, k, v, bl, w["repeat"], w["F"], w["Hl"], w["Wl"], w["n_text"],
+                                          w["stride"], return_lse=True, out_dtype=out_dtype)
+        check_attn(O[:, at["rows"]], at["O_array"])
+        np.testing.assert_allclose(to64(L[:, at["rows"]]), at["LSE_array"], rtol=0, atol=2e-4)
