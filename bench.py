@@ -151,6 +151,33 @@ def _time_calls(fn, steps, warmup, torch):
     return e0.elapsed_time(e1) / steps
 
 
+def _time_graph(fn, calls, torch, replays=5):
+    """Device time per call of a short kernel: `calls` calls captured in one CUDA graph,
+    replayed (after one untimed replay) between events, so that the host's per-call cost
+    is not what gets measured."""
+    fn()
+    torch.cuda.synchronize()
+    side = torch.cuda.Stream()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(g, stream=side):
+            for _ in range(calls):
+                fn()
+    torch.cuda.synchronize()
+    g.replay()
+    torch.cuda.synchronize()
+    st = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(st)
+    for _ in range(replays):
+        g.replay()
+    e1.record(st)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / (replays * calls)
+    del g
+    return ms
+
+
 def cpu_baseline(wl, q, k, v, mask, budget_s: float = 12.0):
     """The float64 oracle on a bounded sample: whole query blocks of head 0 (kept keys only
     enter the softmax), as many as fit in ~budget_s.  Returns kept-only TFLOPS."""
@@ -451,7 +478,7 @@ def main():
             energy = ops.block_energy(q, k, B)
             ms_energy = _time_calls(lambda: ops.block_energy(q, k, B, out=energy), 3, 2, torch)
             msk = torch.empty(energy.shape, dtype=torch.uint8, device=dev)
-            ms_sel = _time_calls(lambda: ops.select_mask(energy, 0.95, out=msk), 20, 3, torch)
+            ms_sel = _time_graph(lambda: ops.select_mask(energy, 0.95, out=msk), 20, torch)
             sel_bytes = energy.numel() * 4 + msk.numel()
             # LSE reuse: a dense forward that emits the row LSE (calibration runs the dense
             # model anyway), then the energy pass with that LSE runs a single pass
@@ -489,9 +516,11 @@ def main():
             # interval form of the default workload's skip list (mask storage)
             rows = H * s.nblk
             iv = ops.csr_to_intervals(bl.row_ptr, bl.col_idx, H, s.nblk)
-            ms_enc = _time_calls(lambda: ops.lib().calib_csr_to_intervals(
+            # the raw ABI call on the current stream (the binding's wrapper reads the run count
+            # back to the host, which a graph capture does not allow)
+            ms_enc = _time_graph(lambda: ops.lib().calib_csr_to_intervals(
                 bl.row_ptr.data_ptr(), bl.col_idx.data_ptr(), H, s.nblk, iv[0].data_ptr(),
-                iv[1].data_ptr(), iv[2].data_ptr(), None), 20, 3, torch)
+                iv[1].data_ptr(), iv[2].data_ptr(), torch.cuda.current_stream().cuda_stream), 20, torch)
             nnz, n_iv = int(bl.row_ptr[-1].item()), int(iv[0][-1].item())
             extras["calibration"]["skip_list_intervals"] = {
                 "kept_blocks": nnz, "runs": n_iv, "blocks_per_run": nnz / max(1, n_iv),

@@ -7,6 +7,7 @@
 
 #include <cmath>
 #include <cstdint>
+#include <type_traits>
 #include <cstring>
 #include <mutex>
 #include <set>
@@ -251,8 +252,17 @@ calib_status calib_select_mask(const float* energy, int H, int nq, int nk, doubl
     if (static_cast<long long>(H) * nq * nk > (1ll << 31) - 1) return CALIB_ERR_INVALID;
     if (calib_status s = check_device()) return s;
     const int rows = H * nq;
-    calib::select_mask_kernel<<<rows_grid(rows), 128, 0, as_stream(stream)>>>(energy, rows, nq, nk, tau, force_keep,
-                                                                               mask_out, count_accum);
+    // energies per lane: the smallest instantiated count covering the row
+    auto launch = [&](auto mpl) {
+        calib::select_mask_kernel<decltype(mpl)::value><<<rows_grid(rows), 128, 0, as_stream(stream)>>>(
+            energy, rows, nq, nk, tau, force_keep, mask_out, count_accum);
+    };
+    if (nk <= 64) launch(std::integral_constant<int, 2>{});
+    else if (nk <= 128) launch(std::integral_constant<int, 4>{});
+    else if (nk <= 256) launch(std::integral_constant<int, 8>{});
+    else if (nk <= 512) launch(std::integral_constant<int, 16>{});
+    else if (nk <= 640) launch(std::integral_constant<int, 20>{});
+    else launch(std::integral_constant<int, 32>{});
     return launch_status();
 }
 
