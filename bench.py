@@ -238,11 +238,21 @@ def run_energy_only(args, wl, dev, torch, ops, synth):
     q, k, _ = synth.make_qkv(wl, device=dev, heads=H)
     E = ops.block_energy(q, k, s.block)
     ms = _time_calls(lambda: ops.block_energy(q, k, s.block, out=E), args.steps, args.warmup, torch)
+    # the selection pass on these energies, with vote-count accumulation (device time)
+    msk = torch.empty(E.shape, dtype=torch.uint8, device=dev)
+    cnt = torch.zeros(E.shape, dtype=torch.int32, device=dev)
+    ms_sel = _time_graph(lambda: ops.select_mask(E, 0.95, out=msk, count_accum=cnt), 20, torch)
     ops.device_check()
     exps = 2.0 * s.N * s.N * H / (ms * 1e-3)
     peak = MUFU_EX2_PER_CLK_SM * B200_SMS * 1965.0e6
+    sel_bytes = E.numel() * (4 + 1 + 4 + 4)       # energies in, mask out, counts read + written
+    hbm = _peaks()["hbm_gbs"]
     print(json.dumps({"leg": "block_energy", "workload": wl.name, "H": H, "N": s.N, "D": s.D, "block": s.block,
-                      "ms": ms, "exp2_per_s": exps, "frac_of_mufu_at_1965mhz": exps / peak}), flush=True)
+                      "ms": ms, "exp2_per_s": exps, "frac_of_mufu_at_1965mhz": exps / peak,
+                      "select": {"shape": list(E.shape), "tau": 0.95, "ms": ms_sel,
+                                 "gbs": sel_bytes / (ms_sel * 1e-3) / 1e9,
+                                 "frac_hbm": sel_bytes / (ms_sel * 1e-3) / 1e9 / hbm,
+                                 "kept_density": float(msk.float().mean().item())}}), flush=True)
 
 
 def run_calibration_sweep(dev, torch, ops, synth):
