@@ -12,6 +12,7 @@
 #include <mutex>
 #include <set>
 #include <utility>
+#include <vector>
 
 #include "calibatt.h"
 #include "ptx.cuh"
@@ -116,9 +117,17 @@ calib_status launch_attn_lse(const CUtensorMap& tk, const CUtensorMap& tv,
     return p.lse ? launch_attn<D, BLK, true>(tk, tv, p, grid, st) : launch_attn<D, BLK, false>(tk, tv, p, grid, st);
 }
 
-calib_status attn_common(const void* q, const void* k, const void* v, void* o, float* lse, int H, int N,
-                         int D, float scale, const calib_block_list* list, const uint32_t* repeat_bits,
-                         int F, int Hl, int Wl, int n_text, int stride, uint32_t flags, void* stream) {
+// A validated attention call: parameters and tensor maps, launchable in slices of the
+// work list.
+struct AttnCall {
+    calib::AttnParams p;
+    CUtensorMap tk, tv;
+    int D, B, grid;
+};
+
+calib_status attn_prepare(const void* q, const void* k, const void* v, void* o, float* lse, int H, int N,
+                          int D, float scale, const calib_block_list* list, const uint32_t* repeat_bits,
+                          int F, int Hl, int Wl, int n_text, int stride, uint32_t flags, AttnCall* c) {
     if (!q || !k || !v || !o || !list || !list->row_ptr || !list->col_idx) return CALIB_ERR_INVALID;
     if (flags & ~CALIB_ATTN_OUT_F32) return CALIB_ERR_INVALID;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return CALIB_ERR_INVALID;
@@ -132,10 +141,9 @@ calib_status attn_common(const void* q, const void* k, const void* v, void* o, f
     if (list->H != H || list->nq != nb || list->nk != nb || nb > 32767 || H > 32767) return CALIB_ERR_INVALID;
     if (list->work && list->n_work < 0) return CALIB_ERR_INVALID;
     if (calib_status s = check_device()) return s;
-    const int grid = list->work ? list->n_work : H * nb;
-    if (grid == 0) return CALIB_OK;
 
-    calib::AttnParams p{};
+    calib::AttnParams& p = c->p;
+    p = calib::AttnParams{};
     p.q = static_cast<const __nv_bfloat16*>(q);
     p.o = static_cast<__nv_bfloat16*>(o);
     p.lse = lse;
@@ -151,14 +159,50 @@ calib_status attn_common(const void* q, const void* k, const void* v, void* o, f
     for (int w = 0; w < 32; ++w) p.repeat_bits[w] = repeat_bits ? repeat_bits[w] : 0u;
     p.out_f32 = (flags & CALIB_ATTN_OUT_F32) ? 1 : 0;
     p.timeout_ns = kDefaultTimeoutNs;
-
-    CUtensorMap tk, tv;
-    if (!make_tmap(&tk, k, D, N, H, B) || !make_tmap(&tv, v, D, N, H, B)) return CALIB_ERR_CUDA;
-    cudaStream_t st = as_stream(stream);
-    if (D == 128) return B == 128 ? launch_attn_lse<128, 128>(tk, tv, p, grid, st)
-                                  : launch_attn_lse<128, 64>(tk, tv, p, grid, st);
-    return B == 128 ? launch_attn_lse<64, 128>(tk, tv, p, grid, st) : launch_attn_lse<64, 64>(tk, tv, p, grid, st);
+    c->D = D;
+    c->B = B;
+    c->grid = list->work ? list->n_work : H * nb;
+    if (!make_tmap(&c->tk, k, D, N, H, B) || !make_tmap(&c->tv, v, D, N, H, B)) return CALIB_ERR_CUDA;
+    return CALIB_OK;
 }
+
+// Launch work items [first, first + count) of a prepared call (items index the work list,
+// which must be present unless the slice is the whole grid).
+calib_status attn_launch(const AttnCall& c, int first, int count, cudaStream_t st) {
+    if (count <= 0) return CALIB_OK;
+    calib::AttnParams p = c.p;
+    if (p.work) p.work += first;
+    else if (first != 0 || count != c.grid) return CALIB_ERR_INVALID;
+    if (c.D == 128) return c.B == 128 ? launch_attn_lse<128, 128>(c.tk, c.tv, p, count, st)
+                                      : launch_attn_lse<128, 64>(c.tk, c.tv, p, count, st);
+    return c.B == 128 ? launch_attn_lse<64, 128>(c.tk, c.tv, p, count, st)
+                      : launch_attn_lse<64, 64>(c.tk, c.tv, p, count, st);
+}
+
+calib_status attn_common(const void* q, const void* k, const void* v, void* o, float* lse, int H, int N,
+                         int D, float scale, const calib_block_list* list, const uint32_t* repeat_bits,
+                         int F, int Hl, int Wl, int n_text, int stride, uint32_t flags, void* stream) {
+    AttnCall c;
+    if (calib_status s = attn_prepare(q, k, v, o, lse, H, N, D, scale, list, repeat_bits, F, Hl, Wl, n_text,
+                                      stride, flags, &c))
+        return s;
+    return attn_launch(c, 0, c.grid, as_stream(stream));
+}
+
+// CUDA events of one call, destroyed on every exit path (a recorded event may be destroyed
+// before it completes; its resources are released once it does).
+struct EventSet {
+    std::vector<cudaEvent_t> ev;
+    cudaEvent_t make() {
+        cudaEvent_t e = nullptr;
+        if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return nullptr;
+        ev.push_back(e);
+        return e;
+    }
+    ~EventSet() {
+        for (cudaEvent_t e : ev) cudaEventDestroy(e);
+    }
+};
 
 // ---- energy ------------------------------------------------------------------------
 template <int D, int BLK>
@@ -392,6 +436,66 @@ calib_status calib_anchor_rows(int F, int Hl, int Wl, int n_text, int stride, in
 calib_status sparse_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse_opt, int H, int N,
                              int D, float scale, const calib_block_list* list, uint32_t flags, void* stream) {
     return attn_common(q, k, v, o, lse_opt, H, N, D, scale, list, nullptr, 1, 1, N, 0, 1, flags, stream);
+}
+
+calib_status sparse_attn_fwd_host(const void* q_host, const void* k_host, const void* v_host, void* o_host,
+                                  void* q_dev, void* k_dev, void* v_dev, void* o_dev, float* lse_opt, int H,
+                                  int N, int D, float scale, const calib_block_list* list, uint32_t flags,
+                                  int heads_per_chunk, void* stream, void* h2d_stream, void* d2h_stream) {
+    if (!q_host || !k_host || !v_host || !o_host || heads_per_chunk < 1) return CALIB_ERR_INVALID;
+    AttnCall c;
+    if (calib_status s = attn_prepare(q_dev, k_dev, v_dev, o_dev, lse_opt, H, N, D, scale, list, nullptr, 1, 1, N,
+                                      0, 1, flags, &c))
+        return s;
+    const int nb = list->nq;
+    // Head chunks need the head-major work order (each head's nq items contiguous, as
+    // calib_build_schedule writes it); any other list runs as one chunk.
+    const bool chunked = list->work && list->n_work == H * nb && heads_per_chunk < H;
+    const int hpc = chunked ? heads_per_chunk : H;
+    const size_t in_head = static_cast<size_t>(N) * D * 2;
+    const size_t out_head = static_cast<size_t>(N) * D * ((flags & CALIB_ATTN_OUT_F32) ? 4 : 2);
+    cudaStream_t st = as_stream(stream);
+    cudaStream_t sin = h2d_stream ? as_stream(h2d_stream) : st;
+    cudaStream_t sout = d2h_stream ? as_stream(d2h_stream) : st;
+    EventSet evs;
+    cudaEvent_t start = evs.make();
+    if (!start || cudaEventRecord(start, st) != cudaSuccess) return CALIB_ERR_CUDA;
+    // the copy streams start after the work already queued on the caller's stream
+    if (cudaStreamWaitEvent(sin, start, 0) != cudaSuccess || cudaStreamWaitEvent(sout, start, 0) != cudaSuccess)
+        return CALIB_ERR_CUDA;
+    auto bytes_at = [](const void* base, size_t off) {
+        return static_cast<const char*>(base) + off;
+    };
+    for (int h0 = 0; h0 < H; h0 += hpc) {
+        const int h1 = h0 + hpc < H ? h0 + hpc : H;
+        const size_t off = static_cast<size_t>(h0) * in_head, len = static_cast<size_t>(h1 - h0) * in_head;
+        // one copy per tensor and chunk
+        if (cudaMemcpyAsync(static_cast<char*>(q_dev) + off, bytes_at(q_host, off), len, cudaMemcpyHostToDevice,
+                            sin) != cudaSuccess ||
+            cudaMemcpyAsync(static_cast<char*>(k_dev) + off, bytes_at(k_host, off), len, cudaMemcpyHostToDevice,
+                            sin) != cudaSuccess ||
+            cudaMemcpyAsync(static_cast<char*>(v_dev) + off, bytes_at(v_host, off), len, cudaMemcpyHostToDevice,
+                            sin) != cudaSuccess)
+            return CALIB_ERR_CUDA;
+        cudaEvent_t in_ready = evs.make();
+        if (!in_ready || cudaEventRecord(in_ready, sin) != cudaSuccess || cudaStreamWaitEvent(st, in_ready, 0) != cudaSuccess)
+            return CALIB_ERR_CUDA;
+        const int first = chunked ? h0 * nb : 0, count = chunked ? (h1 - h0) * nb : c.grid;
+        if (calib_status s = attn_launch(c, first, count, st)) return s;
+        cudaEvent_t out_ready = evs.make();
+        if (!out_ready || cudaEventRecord(out_ready, st) != cudaSuccess ||
+            cudaStreamWaitEvent(sout, out_ready, 0) != cudaSuccess)
+            return CALIB_ERR_CUDA;
+        const size_t ooff = static_cast<size_t>(h0) * out_head, olen = static_cast<size_t>(h1 - h0) * out_head;
+        if (cudaMemcpyAsync(static_cast<char*>(o_host) + ooff, static_cast<const char*>(o_dev) + ooff, olen,
+                            cudaMemcpyDeviceToHost, sout) != cudaSuccess)
+            return CALIB_ERR_CUDA;
+    }
+    // the caller's stream is ordered after the last copy of O
+    cudaEvent_t done = evs.make();
+    if (!done || cudaEventRecord(done, sout) != cudaSuccess || cudaStreamWaitEvent(st, done, 0) != cudaSuccess)
+        return CALIB_ERR_CUDA;
+    return CALIB_OK;
 }
 
 calib_status sparse_attn_fwd_repeat(const void* q, const void* k, const void* v, void* o, float* lse_opt, int H,

@@ -54,6 +54,8 @@ _SIGS = {
                         ctypes.c_int),
     "sparse_attn_fwd_repeat": ([_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _F,
                                 ctypes.POINTER(_BlockListC), _U32, _P], ctypes.c_int),
+    "sparse_attn_fwd_host": ([_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _F, ctypes.POINTER(_BlockListC),
+                              _U32, _I, _P, _P, _P], ctypes.c_int),
     "calib_selftest_wait_timeout": ([_U32, _P], ctypes.c_int),
 }
 
@@ -359,3 +361,74 @@ def sparse_attn_fwd_repeat(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, bl
         _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), H, D, F, Hl, Wl, n_text, stride,
         ctypes.cast(flags, ctypes.c_void_p), scale, ctypes.byref(cs), oflags, _stream()))
     return (out, lse) if (return_lse or lse is not None) else out
+
+
+# ----------------------------------------------------------------------------------
+# inference on host tensors: transfers overlapped with the attention, chunk by chunk
+# ----------------------------------------------------------------------------------
+
+_copy_streams = {}
+
+
+def _side_streams(device: torch.device):
+    """Two copy streams per device (host -> device and device -> host), created once."""
+    key = device.index if device.index is not None else torch.cuda.current_device()
+    if key not in _copy_streams:
+        with torch.cuda.device(key):
+            _copy_streams[key] = (torch.cuda.Stream(), torch.cuda.Stream())
+    return _copy_streams[key]
+
+
+@dataclass
+class HostStaging:
+    """Device staging buffers for sparse_attn_fwd_host: q, k, v bf16 and o [H, N, D]."""
+    q: torch.Tensor
+    k: torch.Tensor
+    v: torch.Tensor
+    o: torch.Tensor
+
+    @staticmethod
+    def allocate(H: int, N: int, D: int, device="cuda", out_dtype: torch.dtype = torch.bfloat16) -> "HostStaging":
+        mk = lambda dt: torch.empty((H, N, D), dtype=dt, device=device)
+        return HostStaging(mk(torch.bfloat16), mk(torch.bfloat16), mk(torch.bfloat16), mk(out_dtype))
+
+
+def sparse_attn_fwd_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, blist: BlockList,
+                         staging: Optional[HostStaging] = None, out: Optional[torch.Tensor] = None,
+                         heads_per_chunk: int = 1, scale: Optional[float] = None,
+                         lse: Optional[torch.Tensor] = None, out_dtype: torch.dtype = torch.bfloat16,
+                         device=None) -> torch.Tensor:
+    """Block-sparse attention of CPU tensors q, k, v (bf16 [H, N, D], pinned for overlap),
+    returning O in a CPU tensor (pinned when allocated here).  The call returns once the
+    work is queued on the current stream; synchronise it before reading O."""
+    H, N, D = q.shape
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        if t.device.type != "cpu":
+            raise ValueError(f"{n} must be a host tensor")
+        if t.dtype != torch.bfloat16 or tuple(t.shape) != (H, N, D) or not t.is_contiguous():
+            raise ValueError(f"{n} must be contiguous bf16 [H, N, D]")
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    if staging is None:
+        staging = HostStaging.allocate(H, N, D, dev, out_dtype)
+    out_dtype = staging.o.dtype
+    for t, n in ((staging.q, "staging.q"), (staging.k, "staging.k"), (staging.v, "staging.v")):
+        _need(t, n, torch.bfloat16, (H, N, D))
+    _need(staging.o, "staging.o", out_dtype, (H, N, D))
+    if out_dtype not in (torch.bfloat16, torch.float32):
+        raise TypeError("out must be bf16 or fp32")
+    if out is None:
+        out = torch.empty((H, N, D), dtype=out_dtype, pin_memory=True)
+    if out.device.type != "cpu" or out.dtype != out_dtype or tuple(out.shape) != (H, N, D) or not out.is_contiguous():
+        raise ValueError("out must be a contiguous host tensor of the output dtype and shape")
+    if lse is not None:
+        _need(lse, "lse", torch.float32, (H, N))
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    h2d, d2h = _side_streams(staging.q.device)
+    cs = blist.c_struct()
+    flags = CALIB_ATTN_OUT_F32 if out_dtype == torch.float32 else 0
+    _check("sparse_attn_fwd_host", lib().sparse_attn_fwd_host(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), _ptr(staging.q), _ptr(staging.k),
+        _ptr(staging.v), _ptr(staging.o), _ptr(lse), H, N, D, scale, ctypes.byref(cs), flags,
+        int(heads_per_chunk), _stream(), h2d.cuda_stream, d2h.cuda_stream))
+    return out
+

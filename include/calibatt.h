@@ -209,6 +209,30 @@ calib_status sparse_attn_fwd(const void* q, const void* k, const void* v, void* 
                              float* lse_opt, int H, int N, int D, float scale,
                              const calib_block_list* list, uint32_t flags, void* stream);
 
+/* sparse_attn_fwd on HOST tensors, with the transfers overlapped with the attention: the
+ * heads are processed in chunks of heads_per_chunk; chunk c's Q/K/V go host -> device on
+ * h2d_stream while the kernel of chunk c-1 runs on `stream`, and each chunk's O goes
+ * device -> host on d2h_stream once its kernel is done.
+ *   q_host, k_host, v_host : bf16 [H, N, D] in host memory (page-locked for the copies to
+ *                overlap; pageable memory gives the same result without overlap).
+ *   o_host     : host [H, N, D], bf16 (fp32 with CALIB_ATTN_OUT_F32).
+ *   q_dev, k_dev, v_dev, o_dev : caller-owned device buffers of the same shapes, used as
+ *                staging; their previous contents are overwritten.
+ *   lse_opt    : NULL or a DEVICE fp32 [H, N] buffer (it stays on the device).
+ *   heads_per_chunk >= 1.  Chunks follow the work list, which must then hold each head's nq
+ *                items contiguously in head order (as calib_build_schedule writes it);
+ *                with list->work == NULL or n_work != H*nq the call runs as one chunk.
+ *   h2d_stream, d2h_stream : copy streams (NULL: `stream`, no overlap).
+ * Ordering: the copies start after the work already queued on `stream`, and `stream` is
+ * ordered after the last copy of O, so synchronising `stream` makes o_host complete.
+ * Other arguments, results and errors as sparse_attn_fwd; host pointers must be non-NULL.
+ * The copies are one cudaMemcpyAsync per tensor and chunk. */
+calib_status sparse_attn_fwd_host(const void* q_host, const void* k_host, const void* v_host, void* o_host,
+                                  void* q_dev, void* k_dev, void* v_dev, void* o_dev, float* lse_opt,
+                                  int H, int N, int D, float scale, const calib_block_list* list,
+                                  uint32_t flags, int heads_per_chunk, void* stream, void* h2d_stream,
+                                  void* d2h_stream);
+
 /* Block-sparse attention with spatial repetition ([zh] §2.2B, [fr] §2.C): heads flagged
  * in head_repeat (HOST uint8 [H]) compute only their anchor tokens (calib_anchor_rows
  * order) and write each anchor's output (and LSE) to every token it stands for -- token

@@ -73,6 +73,16 @@ def test_invalid_arguments_rejected_before_device_work():
     # unknown flag bits
     assert L.sparse_attn_fwd(fake, fake, fake, fake, null, 1, 128, 128, 0.1, ctypes.byref(bl), 6, null) == \
         ops.CALIB_ERR_INVALID
+    # host-buffer attention: null host pointers, a chunk size below 1, then the device
+    # buffers' checks (head dim, list shape)
+    assert L.sparse_attn_fwd_host(null, fake, fake, fake, fake, fake, fake, fake, null, 1, 128, 128, 0.1,
+                                  ctypes.byref(bl), 0, 1, null, null, null) == ops.CALIB_ERR_INVALID
+    assert L.sparse_attn_fwd_host(fake, fake, fake, fake, fake, fake, fake, fake, null, 1, 128, 128, 0.1,
+                                  ctypes.byref(bl), 0, 0, null, null, null) == ops.CALIB_ERR_INVALID
+    assert L.sparse_attn_fwd_host(fake, fake, fake, fake, fake, fake, fake, fake, null, 1, 128, 96, 0.1,
+                                  ctypes.byref(bl), 0, 1, null, null, null) == ops.CALIB_ERR_UNSUPPORTED
+    assert L.sparse_attn_fwd_host(fake, fake, fake, fake, fake, fake, fake, fake, null, 1, 128, 128, 0.1,
+                                  ctypes.byref(bl2), 0, 1, null, null, null) == ops.CALIB_ERR_INVALID
     # selection beyond nk = 1024 is unsupported
     assert L.calib_select_mask(fake, 1, 1, 1025, 0.9, null, fake, null, null) in (
         ops.CALIB_ERR_UNSUPPORTED,)
