@@ -481,19 +481,16 @@ def main():
         if world > 1:
             ms_serial = max_over_ranks(ms_serial, dist, dev)
         nb = q.numel() * q.element_size()
-        if any(rep):
-            # the host-buffer entry point covers the plain path; repeat heads copy serially
-            ms_e2e, mode, hpc = ms_serial, "serial copies around sparse_attn_fwd_repeat", None
-        else:
-            # sparse_attn_fwd_host: per chunk of 2 heads, the host -> device copies of the next
-            # chunk and the device -> host copy of the previous one overlap the attention
-            hpc = 2
-            staging = ops.HostStaging(qd, kd, vd, out)
-            ms_e2e = _time_calls(lambda: ops.sparse_attn_fwd_host(qh, kh, vh, bl, staging=staging, out=oh,
-                                                                  heads_per_chunk=hpc), 10, 3, torch)
-            if world > 1:
-                ms_e2e = max_over_ranks(ms_e2e, dist, dev)
-            mode = "sparse_attn_fwd_host: copies overlapped with the attention per head chunk"
+        # sparse_attn_fwd_host: per chunk of 2 heads, the host -> device copies of the next
+        # chunk and the device -> host copy of the previous one overlap the attention
+        hpc = 2
+        staging = ops.HostStaging(qd, kd, vd, out)
+        geom = (rep, s.F, s.Hl, s.Wl, s.n_text, stride) if any(rep) else None
+        ms_e2e = _time_calls(lambda: ops.sparse_attn_fwd_host(qh, kh, vh, bl, staging=staging, out=oh,
+                                                              heads_per_chunk=hpc, repeat=geom), 10, 3, torch)
+        if world > 1:
+            ms_e2e = max_over_ranks(ms_e2e, dist, dev)
+        mode = "sparse_attn_fwd_host: copies overlapped with the attention per head chunk"
         extras["e2e"] = {"value": flops_kept * world / (ms_e2e * 1e-3) / 1e12, "unit": UNIT,
                          "h2d_bytes_per_step": 3 * nb, "d2h_bytes_per_step": nb, "ms_per_step": ms_e2e,
                          "mode": mode, "heads_per_chunk": hpc,

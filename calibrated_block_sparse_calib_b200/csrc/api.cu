@@ -204,6 +204,75 @@ struct EventSet {
     }
 };
 
+// Host <-> device transfers of a prepared attention call, overlapped with its kernels per
+// chunk of heads (see sparse_attn_fwd_host in calibatt.h).
+calib_status host_pipeline(const AttnCall& c, const void* q_host, const void* k_host, const void* v_host,
+                           void* o_host, void* q_dev, void* k_dev, void* v_dev, const void* o_dev, int H, int N,
+                           int D, const calib_block_list* list, uint32_t flags, int heads_per_chunk,
+                           void* stream, void* h2d_stream, void* d2h_stream) {
+    const int nb = list->nq;
+    // Head chunks need the head-major work order (each head's nq items contiguous, as
+    // calib_build_schedule writes it); any other list runs as one chunk.
+    const bool chunked = list->work && list->n_work == H * nb && heads_per_chunk < H;
+    const int hpc = chunked ? heads_per_chunk : H;
+    const size_t in_head = static_cast<size_t>(N) * D * 2;
+    const size_t out_head = static_cast<size_t>(N) * D * ((flags & CALIB_ATTN_OUT_F32) ? 4 : 2);
+    cudaStream_t st = as_stream(stream);
+    cudaStream_t sin = h2d_stream ? as_stream(h2d_stream) : st;
+    cudaStream_t sout = d2h_stream ? as_stream(d2h_stream) : st;
+    EventSet evs;
+    cudaEvent_t start = evs.make();
+    if (!start || cudaEventRecord(start, st) != cudaSuccess) return CALIB_ERR_CUDA;
+    // the copy streams start after the work already queued on the caller's stream
+    if (cudaStreamWaitEvent(sin, start, 0) != cudaSuccess || cudaStreamWaitEvent(sout, start, 0) != cudaSuccess)
+        return CALIB_ERR_CUDA;
+    for (int h0 = 0; h0 < H; h0 += hpc) {
+        const int h1 = h0 + hpc < H ? h0 + hpc : H;
+        const size_t off = static_cast<size_t>(h0) * in_head, len = static_cast<size_t>(h1 - h0) * in_head;
+        // one copy per tensor and chunk
+        if (cudaMemcpyAsync(static_cast<char*>(q_dev) + off, static_cast<const char*>(q_host) + off, len,
+                            cudaMemcpyHostToDevice, sin) != cudaSuccess ||
+            cudaMemcpyAsync(static_cast<char*>(k_dev) + off, static_cast<const char*>(k_host) + off, len,
+                            cudaMemcpyHostToDevice, sin) != cudaSuccess ||
+            cudaMemcpyAsync(static_cast<char*>(v_dev) + off, static_cast<const char*>(v_host) + off, len,
+                            cudaMemcpyHostToDevice, sin) != cudaSuccess)
+            return CALIB_ERR_CUDA;
+        cudaEvent_t in_ready = evs.make();
+        if (!in_ready || cudaEventRecord(in_ready, sin) != cudaSuccess ||
+            cudaStreamWaitEvent(st, in_ready, 0) != cudaSuccess)
+            return CALIB_ERR_CUDA;
+        const int first = chunked ? h0 * nb : 0, count = chunked ? (h1 - h0) * nb : c.grid;
+        if (calib_status s = attn_launch(c, first, count, st)) return s;
+        cudaEvent_t out_ready = evs.make();
+        if (!out_ready || cudaEventRecord(out_ready, st) != cudaSuccess ||
+            cudaStreamWaitEvent(sout, out_ready, 0) != cudaSuccess)
+            return CALIB_ERR_CUDA;
+        const size_t ooff = static_cast<size_t>(h0) * out_head, olen = static_cast<size_t>(h1 - h0) * out_head;
+        if (cudaMemcpyAsync(static_cast<char*>(o_host) + ooff, static_cast<const char*>(o_dev) + ooff, olen,
+                            cudaMemcpyDeviceToHost, sout) != cudaSuccess)
+            return CALIB_ERR_CUDA;
+    }
+    // the caller's stream is ordered after the last copy of O
+    cudaEvent_t done = evs.make();
+    if (!done || cudaEventRecord(done, sout) != cudaSuccess || cudaStreamWaitEvent(st, done, 0) != cudaSuccess)
+        return CALIB_ERR_CUDA;
+    return CALIB_OK;
+}
+
+// Validated repeat geometry: token count N = F*Hl*Wl + n_text and the head bit set.
+calib_status repeat_geometry(int H, int F, int Hl, int Wl, int n_text, int stride, const uint8_t* head_repeat,
+                             uint32_t* bits, int* N_out) {
+    if (!head_repeat || calib_anchor_count(F, Hl, Wl, n_text, stride) < 0 || H < 1 || H > 1024)
+        return CALIB_ERR_INVALID;
+    const long long N = static_cast<long long>(F) * Hl * Wl + n_text;
+    if (N > (1ll << 31) - 1) return CALIB_ERR_INVALID;
+    for (int w = 0; w < 32; ++w) bits[w] = 0u;
+    for (int h = 0; h < H; ++h)
+        if (head_repeat[h]) bits[h >> 5] |= 1u << (h & 31);
+    *N_out = static_cast<int>(N);
+    return CALIB_OK;
+}
+
 // ---- energy ------------------------------------------------------------------------
 template <int D, int BLK>
 calib_status launch_energy(const CUtensorMap& tk, const calib::EnergyParams& p, int grid, cudaStream_t st) {
@@ -447,70 +516,36 @@ calib_status sparse_attn_fwd_host(const void* q_host, const void* k_host, const 
     if (calib_status s = attn_prepare(q_dev, k_dev, v_dev, o_dev, lse_opt, H, N, D, scale, list, nullptr, 1, 1, N,
                                       0, 1, flags, &c))
         return s;
-    const int nb = list->nq;
-    // Head chunks need the head-major work order (each head's nq items contiguous, as
-    // calib_build_schedule writes it); any other list runs as one chunk.
-    const bool chunked = list->work && list->n_work == H * nb && heads_per_chunk < H;
-    const int hpc = chunked ? heads_per_chunk : H;
-    const size_t in_head = static_cast<size_t>(N) * D * 2;
-    const size_t out_head = static_cast<size_t>(N) * D * ((flags & CALIB_ATTN_OUT_F32) ? 4 : 2);
-    cudaStream_t st = as_stream(stream);
-    cudaStream_t sin = h2d_stream ? as_stream(h2d_stream) : st;
-    cudaStream_t sout = d2h_stream ? as_stream(d2h_stream) : st;
-    EventSet evs;
-    cudaEvent_t start = evs.make();
-    if (!start || cudaEventRecord(start, st) != cudaSuccess) return CALIB_ERR_CUDA;
-    // the copy streams start after the work already queued on the caller's stream
-    if (cudaStreamWaitEvent(sin, start, 0) != cudaSuccess || cudaStreamWaitEvent(sout, start, 0) != cudaSuccess)
-        return CALIB_ERR_CUDA;
-    auto bytes_at = [](const void* base, size_t off) {
-        return static_cast<const char*>(base) + off;
-    };
-    for (int h0 = 0; h0 < H; h0 += hpc) {
-        const int h1 = h0 + hpc < H ? h0 + hpc : H;
-        const size_t off = static_cast<size_t>(h0) * in_head, len = static_cast<size_t>(h1 - h0) * in_head;
-        // one copy per tensor and chunk
-        if (cudaMemcpyAsync(static_cast<char*>(q_dev) + off, bytes_at(q_host, off), len, cudaMemcpyHostToDevice,
-                            sin) != cudaSuccess ||
-            cudaMemcpyAsync(static_cast<char*>(k_dev) + off, bytes_at(k_host, off), len, cudaMemcpyHostToDevice,
-                            sin) != cudaSuccess ||
-            cudaMemcpyAsync(static_cast<char*>(v_dev) + off, bytes_at(v_host, off), len, cudaMemcpyHostToDevice,
-                            sin) != cudaSuccess)
-            return CALIB_ERR_CUDA;
-        cudaEvent_t in_ready = evs.make();
-        if (!in_ready || cudaEventRecord(in_ready, sin) != cudaSuccess || cudaStreamWaitEvent(st, in_ready, 0) != cudaSuccess)
-            return CALIB_ERR_CUDA;
-        const int first = chunked ? h0 * nb : 0, count = chunked ? (h1 - h0) * nb : c.grid;
-        if (calib_status s = attn_launch(c, first, count, st)) return s;
-        cudaEvent_t out_ready = evs.make();
-        if (!out_ready || cudaEventRecord(out_ready, st) != cudaSuccess ||
-            cudaStreamWaitEvent(sout, out_ready, 0) != cudaSuccess)
-            return CALIB_ERR_CUDA;
-        const size_t ooff = static_cast<size_t>(h0) * out_head, olen = static_cast<size_t>(h1 - h0) * out_head;
-        if (cudaMemcpyAsync(static_cast<char*>(o_host) + ooff, static_cast<const char*>(o_dev) + ooff, olen,
-                            cudaMemcpyDeviceToHost, sout) != cudaSuccess)
-            return CALIB_ERR_CUDA;
-    }
-    // the caller's stream is ordered after the last copy of O
-    cudaEvent_t done = evs.make();
-    if (!done || cudaEventRecord(done, sout) != cudaSuccess || cudaStreamWaitEvent(st, done, 0) != cudaSuccess)
-        return CALIB_ERR_CUDA;
-    return CALIB_OK;
+    return host_pipeline(c, q_host, k_host, v_host, o_host, q_dev, k_dev, v_dev, o_dev, H, N, D, list, flags,
+                         heads_per_chunk, stream, h2d_stream, d2h_stream);
+}
+
+calib_status sparse_attn_fwd_repeat_host(const void* q_host, const void* k_host, const void* v_host,
+                                         void* o_host, void* q_dev, void* k_dev, void* v_dev, void* o_dev,
+                                         float* lse_opt, int H, int D, int F, int Hl, int Wl, int n_text,
+                                         int stride, const uint8_t* head_repeat, float scale,
+                                         const calib_block_list* list, uint32_t flags, int heads_per_chunk,
+                                         void* stream, void* h2d_stream, void* d2h_stream) {
+    if (!q_host || !k_host || !v_host || !o_host || heads_per_chunk < 1) return CALIB_ERR_INVALID;
+    uint32_t bits[32];
+    int N = 0;
+    if (calib_status s = repeat_geometry(H, F, Hl, Wl, n_text, stride, head_repeat, bits, &N)) return s;
+    AttnCall c;
+    if (calib_status s = attn_prepare(q_dev, k_dev, v_dev, o_dev, lse_opt, H, N, D, scale, list, bits, F, Hl, Wl,
+                                      n_text, stride, flags, &c))
+        return s;
+    return host_pipeline(c, q_host, k_host, v_host, o_host, q_dev, k_dev, v_dev, o_dev, H, N, D, list, flags,
+                         heads_per_chunk, stream, h2d_stream, d2h_stream);
 }
 
 calib_status sparse_attn_fwd_repeat(const void* q, const void* k, const void* v, void* o, float* lse_opt, int H,
                                     int D, int F, int Hl, int Wl, int n_text, int stride,
                                     const uint8_t* head_repeat, float scale, const calib_block_list* list,
                                     uint32_t flags, void* stream) {
-    if (!head_repeat || calib_anchor_count(F, Hl, Wl, n_text, stride) < 0 || H < 1 || H > 1024)
-        return CALIB_ERR_INVALID;
-    const long long N = static_cast<long long>(F) * Hl * Wl + n_text;
-    if (N > (1ll << 31) - 1) return CALIB_ERR_INVALID;
-    uint32_t bits[32] = {0};
-    for (int h = 0; h < H; ++h)
-        if (head_repeat[h]) bits[h >> 5] |= 1u << (h & 31);
-    return attn_common(q, k, v, o, lse_opt, H, static_cast<int>(N), D, scale, list, bits, F, Hl, Wl, n_text,
-                       stride, flags, stream);
+    uint32_t bits[32];
+    int N = 0;
+    if (calib_status s = repeat_geometry(H, F, Hl, Wl, n_text, stride, head_repeat, bits, &N)) return s;
+    return attn_common(q, k, v, o, lse_opt, H, N, D, scale, list, bits, F, Hl, Wl, n_text, stride, flags, stream);
 }
 
 calib_status calib_selftest_wait_timeout(uint32_t timeout_us, void* stream) {

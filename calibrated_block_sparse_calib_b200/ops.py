@@ -56,6 +56,8 @@ _SIGS = {
                                 ctypes.POINTER(_BlockListC), _U32, _P], ctypes.c_int),
     "sparse_attn_fwd_host": ([_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _F, ctypes.POINTER(_BlockListC),
                               _U32, _I, _P, _P, _P], ctypes.c_int),
+    "sparse_attn_fwd_repeat_host": ([_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _F,
+                                     ctypes.POINTER(_BlockListC), _U32, _I, _P, _P, _P], ctypes.c_int),
     "calib_selftest_wait_timeout": ([_U32, _P], ctypes.c_int),
 }
 
@@ -397,10 +399,11 @@ def sparse_attn_fwd_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, blis
                          staging: Optional[HostStaging] = None, out: Optional[torch.Tensor] = None,
                          heads_per_chunk: int = 1, scale: Optional[float] = None,
                          lse: Optional[torch.Tensor] = None, out_dtype: torch.dtype = torch.bfloat16,
-                         device=None) -> torch.Tensor:
+                         device=None, repeat: Optional[tuple] = None) -> torch.Tensor:
     """Block-sparse attention of CPU tensors q, k, v (bf16 [H, N, D], pinned for overlap),
     returning O in a CPU tensor (pinned when allocated here).  The call returns once the
-    work is queued on the current stream; synchronise it before reading O."""
+    work is queued on the current stream; synchronise it before reading O.
+    repeat = (head_repeat, F, Hl, Wl, n_text, stride) selects spatial-repetition mode."""
     H, N, D = q.shape
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         if t.device.type != "cpu":
@@ -426,9 +429,20 @@ def sparse_attn_fwd_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, blis
     h2d, d2h = _side_streams(staging.q.device)
     cs = blist.c_struct()
     flags = CALIB_ATTN_OUT_F32 if out_dtype == torch.float32 else 0
-    _check("sparse_attn_fwd_host", lib().sparse_attn_fwd_host(
+    if repeat is None:
+        _check("sparse_attn_fwd_host", lib().sparse_attn_fwd_host(
+            q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), _ptr(staging.q), _ptr(staging.k),
+            _ptr(staging.v), _ptr(staging.o), _ptr(lse), H, N, D, scale, ctypes.byref(cs), flags,
+            int(heads_per_chunk), _stream(), h2d.cuda_stream, d2h.cuda_stream))
+        return out
+    head_repeat, F, Hl, Wl, n_text, stride = repeat
+    if N != F * Hl * Wl + n_text:
+        raise ValueError("N must equal F*Hl*Wl + n_text")
+    rflags = (ctypes.c_uint8 * H)(*[1 if bool(x) else 0 for x in head_repeat])
+    _check("sparse_attn_fwd_repeat_host", lib().sparse_attn_fwd_repeat_host(
         q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), _ptr(staging.q), _ptr(staging.k),
-        _ptr(staging.v), _ptr(staging.o), _ptr(lse), H, N, D, scale, ctypes.byref(cs), flags,
-        int(heads_per_chunk), _stream(), h2d.cuda_stream, d2h.cuda_stream))
+        _ptr(staging.v), _ptr(staging.o), _ptr(lse), H, D, F, Hl, Wl, n_text, stride,
+        ctypes.cast(rflags, ctypes.c_void_p), scale, ctypes.byref(cs), flags, int(heads_per_chunk), _stream(),
+        h2d.cuda_stream, d2h.cuda_stream))
     return out
 

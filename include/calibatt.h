@@ -233,6 +233,17 @@ calib_status sparse_attn_fwd_host(const void* q_host, const void* k_host, const 
                                   uint32_t flags, int heads_per_chunk, void* stream, void* h2d_stream,
                                   void* d2h_stream);
 
+/* sparse_attn_fwd_repeat on HOST tensors, transfers overlapped per head chunk as in
+ * sparse_attn_fwd_host (a repeat head's broadcast stays inside its own head, so chunks of
+ * heads are independent).  Repeat arguments as sparse_attn_fwd_repeat; host, staging,
+ * chunk and stream arguments as sparse_attn_fwd_host. */
+calib_status sparse_attn_fwd_repeat_host(const void* q_host, const void* k_host, const void* v_host,
+                                         void* o_host, void* q_dev, void* k_dev, void* v_dev, void* o_dev,
+                                         float* lse_opt, int H, int D, int F, int Hl, int Wl, int n_text,
+                                         int stride, const uint8_t* head_repeat, float scale,
+                                         const calib_block_list* list, uint32_t flags, int heads_per_chunk,
+                                         void* stream, void* h2d_stream, void* d2h_stream);
+
 /* Block-sparse attention with spatial repetition ([zh] §2.2B, [fr] §2.C): heads flagged
  * in head_repeat (HOST uint8 [H]) compute only their anchor tokens (calib_anchor_rows
  * order) and write each anchor's output (and LSE) to every token it stands for -- token

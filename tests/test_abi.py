@@ -83,6 +83,13 @@ def test_invalid_arguments_rejected_before_device_work():
                                   ctypes.byref(bl), 0, 1, null, null, null) == ops.CALIB_ERR_UNSUPPORTED
     assert L.sparse_attn_fwd_host(fake, fake, fake, fake, fake, fake, fake, fake, null, 1, 128, 128, 0.1,
                                   ctypes.byref(bl2), 0, 1, null, null, null) == ops.CALIB_ERR_INVALID
+    rep = (ctypes.c_uint8 * 1)(1)
+    assert L.sparse_attn_fwd_repeat_host(null, fake, fake, fake, fake, fake, fake, fake, null, 1, 128, 1, 1, 128,
+                                         0, 1, ctypes.cast(rep, ctypes.c_void_p), 0.1, ctypes.byref(bl), 0, 1,
+                                         null, null, null) == ops.CALIB_ERR_INVALID
+    assert L.sparse_attn_fwd_repeat_host(fake, fake, fake, fake, fake, fake, fake, fake, null, 1, 128, 1, 1, 128,
+                                         0, 1, null, 0.1, ctypes.byref(bl), 0, 1, null, null,
+                                         null) == ops.CALIB_ERR_INVALID
     # selection beyond nk = 1024 is unsupported
     assert L.calib_select_mask(fake, 1, 1, 1025, 0.9, null, fake, null, null) in (
         ops.CALIB_ERR_UNSUPPORTED,)

@@ -802,3 +802,29 @@ def test_host_io_attention_back_to_back_calls_reuse_staging():
     torch.cuda.current_stream().synchronize()
     assert torch.equal(oa, ops.sparse_attn_fwd(*(t.cuda() for t in a), bl).cpu())
     assert torch.equal(ob, ops.sparse_attn_fwd(*(t.cuda() for t in b), bl).cpu())
+
+
+@pytest.mark.parametrize("hpc", [1, 2, 3])
+def test_host_io_repeat_attention_equals_device_call(hpc):
+    """Spatial-repetition mode through host buffers (text tokens, ragged anchor groups,
+    two of three heads flagged): O and LSE equal the device-resident call bit for bit."""
+    wl = _shape(3, 128, 3, 7, 20, 128, n_text=40)
+    s = wl.shape
+    stride = 3
+    q, k, v = synth.make_qkv(wl, seed=77)
+    nb = s.nblk
+    m = _rand_mask(np.random.default_rng(78), 3, nb, nb, 0.5)
+    nqa = synth.anchor_block_count(s, stride)
+    rep = [True, False, True]
+    for h in (0, 2):
+        m[h, nqa:] = 0
+    bl = _blist(m, 128)
+    geom = (rep, s.F, s.Hl, s.Wl, s.n_text, stride)
+    lse_h = torch.empty(s.H, s.N, dtype=torch.float32, device="cuda")
+    o_host = ops.sparse_attn_fwd_host(*(t.contiguous().pin_memory() for t in (q, k, v)), bl, heads_per_chunk=hpc,
+                                      lse=lse_h, repeat=geom)
+    torch.cuda.current_stream().synchronize()
+    O_dev, L_dev = ops.sparse_attn_fwd_repeat(q.cuda(), k.cuda(), v.cuda(), bl, *geom, return_lse=True)
+    torch.cuda.synchronize()
+    assert torch.equal(o_host, O_dev.cpu())
+    assert torch.equal(lse_h.cpu(), L_dev.cpu())
