@@ -556,7 +556,8 @@ def main():
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": wl.name, "H": H, "N": N, "D": D, "block": B, "density": round(density, 4),
                    "repeat_heads": sum(rep), "parallelism": f"replicas{world}",
-                   "l2": "inputs larger than L2 (Q/K/V/O 403 MB), no flush"},
+                   "l2": f"inputs larger than L2 (Q/K/V/O {4 * q.numel() * q.element_size() / 1e6:.0f} MB), "
+                         "no flush"},
         "dense_equiv_tflops": flops_dense * world / (ms * 1e-3) / 1e12,
         "frac_of_bf16_peak": value / world / peaks["bf16_tflops"],
         "roofline": {"bound": "tensor", "achieved": value / world, "peak": peaks["bf16_tflops"],
