@@ -37,8 +37,9 @@ METRIC = "sparse attn TFLOPS (kept-only & dense-equiv) + % BF16 TC peak at 30% d
 UNIT = "TFLOPS"
 
 # DRAM bytes (read + write) of one attn_fwd_kernel launch on the wan13b workload, from an
-# ncu capture (profiles/attn_fwd_wan13b.md), valid only for the kernel sources it was taken
-# on: reported as roofline.traffic while the source hashes still match, else null.
+# ncu capture of that launch (dram__bytes_read.sum + dram__bytes_write.sum), valid only for
+# the kernel sources it was taken on: reported as roofline.traffic while the source hashes
+# still match, else null.
 NCU_TRAFFIC = {("wan13b", "dbf78f98d8d3", "14017e6adac8"): 302_587_904 + 87_381_504}
 
 # MUFU exp2 throughput of one SM: 4 lanes per clock in each of the 4 sub-partitions.
