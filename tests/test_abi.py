@@ -96,3 +96,22 @@ def test_invalid_arguments_rejected_before_device_work():
     # energy pass beyond N = 131072 tokens is unsupported
     assert L.calib_block_energy(fake, fake, null, 1, 131073, 128, 128, 0.1, null, 0, fake, 0, null) == \
         ops.CALIB_ERR_UNSUPPORTED
+
+
+def test_plain_c_client(tmp_path):
+    """The header compiles as C99 and a C program linked to the library gets the documented
+    answers from the host-decided paths (tests/abi_client.c), with no Python in between."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("gcc not available")
+    ops.lib()                                          # the library exists (built in-tree)
+    libdir = os.path.dirname(ops.LIB_PATH)
+    exe = str(tmp_path / "abi_client")
+    cmd = [gcc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-I", os.path.join(ROOT, "include"),
+           os.path.join(ROOT, "tests", "abi_client.c"), "-L", libdir, "-lcalibatt", f"-Wl,-rpath,{libdir}",
+           "-o", exe]
+    subprocess.run(cmd, check=True, capture_output=True, text=True)
+    res = subprocess.run([exe], capture_output=True, text=True, timeout=120)
+    assert res.returncode == 0 and res.stdout.strip() == "ok", res.stdout + res.stderr
