@@ -115,3 +115,27 @@ def test_plain_c_client(tmp_path):
     subprocess.run(cmd, check=True, capture_output=True, text=True)
     res = subprocess.run([exe], capture_output=True, text=True, timeout=120)
     assert res.returncode == 0 and res.stdout.strip() == "ok", res.stdout + res.stderr
+
+
+def test_product_path_refuses_host_tensors_and_a_missing_library(monkeypatch):
+    """No CPU fallback: device entry points reject CPU tensors before any call, and a
+    missing shared library raises instead of degrading to another implementation."""
+    import torch
+    q = torch.zeros(1, 128, 128, dtype=torch.bfloat16)
+    m = torch.ones(1, 1, 1, dtype=torch.uint8)
+    bl = ops.BlockList(1, 1, 1, 128, torch.zeros(2, dtype=torch.int32), torch.zeros(1, dtype=torch.int16))
+    with pytest.raises(TypeError, match="CUDA tensor"):
+        ops.sparse_attn_fwd(q, q, q, bl)
+    with pytest.raises(TypeError, match="CUDA tensor"):
+        ops.block_energy(q, q, 128)
+    with pytest.raises(TypeError, match="CUDA tensor"):
+        ops.select_mask(torch.zeros(1, 1, 1), 0.9)
+    with pytest.raises(TypeError, match="CUDA tensor"):
+        ops.mask_to_csr(m)
+    if not torch.cuda.is_available():
+        with pytest.raises(Exception):
+            ops.sparse_attn_fwd_host(q, q, q, bl)       # needs a device for its staging buffers
+    monkeypatch.setattr(ops, "_lib", None)
+    monkeypatch.setattr(ops, "LIB_PATH", os.path.join(ROOT, "no_such_dir", "libcalibatt.so"))
+    with pytest.raises(RuntimeError, match="missing"):
+        ops.lib()
