@@ -226,6 +226,8 @@ calib_status sparse_attn_fwd(const void* q, const void* k, const void* v, void* 
  * Ordering: the copies start after the work already queued on `stream`, and `stream` is
  * ordered after the last copy of O, so synchronising `stream` makes o_host complete.
  * Other arguments, results and errors as sparse_attn_fwd; host pointers must be non-NULL.
+ * Argument errors are reported before anything is enqueued; a CUDA error met while
+ * enqueueing (CALIB_ERR_CUDA) can leave the earlier chunks' copies and kernels queued.
  * The copies are one cudaMemcpyAsync per tensor and chunk. */
 calib_status sparse_attn_fwd_host(const void* q_host, const void* k_host, const void* v_host, void* o_host,
                                   void* q_dev, void* k_dev, void* v_dev, void* o_dev, float* lse_opt,
