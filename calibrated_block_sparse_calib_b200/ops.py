@@ -426,6 +426,8 @@ def sparse_attn_fwd_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, blis
     if lse is not None:
         _need(lse, "lse", torch.float32, (H, N))
     scale = 1.0 / math.sqrt(D) if scale is None else scale
+    if staging.q.device.index != torch.cuda.current_device():
+        raise ValueError("the staging buffers must be on the current CUDA device")
     h2d, d2h = _side_streams(staging.q.device)
     cs = blist.c_struct()
     flags = CALIB_ATTN_OUT_F32 if out_dtype == torch.float32 else 0
