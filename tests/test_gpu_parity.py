@@ -235,6 +235,29 @@ def test_energy_ragged(D, B, geom):
     check_energy(got, ref, wl.shape.N, B)
 
 
+@pytest.mark.parametrize("geom", [(32, 64, 64, 0), (31, 64, 64, 4095)])
+def test_energy_at_the_maximum_length(geom):
+    """N = 131072 tokens, the longest sequence the energy pass accepts, and 131071 (a
+    ragged last key block of 127 tokens): sampled query blocks against the oracle."""
+    F, Hl, Wl, n_text = geom
+    wl = _shape(1, 128, F, Hl, Wl, 128, n_text=n_text)
+    s = wl.shape
+    assert s.N in (131072, 131071)
+    q, k, _ = synth.make_qkv(wl, seed=900 + n_text)
+    got = ops.block_energy(q.cuda(), k.cuda(), 128).cpu()
+    blocks = [0, 517, s.nblk - 1]
+    ref = oracle.block_energy(to64(q), to64(k), 1.0 / math.sqrt(128), 128, q_blocks=blocks)
+    g = to64(got)[:, blocks]
+    rows = np.array([min((i + 1) * 128, s.N) - i * 128 for i in blocks], float)[None, :, None]
+    big = ref >= 1e-12 * rows
+    err = np.abs(g - ref)
+    assert np.all(err[big] <= E_REL * ref[big]), float((err[big] / ref[big]).max())
+    assert np.all(err[~big] <= 1e-16 * np.broadcast_to(rows, ref.shape)[~big])
+    # every query row's energies sum to one softmax row
+    np.testing.assert_allclose(to64(got).sum(axis=2)[0], [min((i + 1) * 128, s.N) - i * 128 for i in range(s.nblk)],
+                               rtol=1e-4)
+
+
 def test_energy_cached_lse_and_accumulate(tiny_inputs):
     wl, qkv = tiny_inputs
     B, D = wl.shape.block, wl.shape.D
