@@ -14,6 +14,14 @@ def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
 
 
+def pytest_sessionstart(session):
+    """A fresh checkout has no libcalibatt.so (built files are not versioned): build it
+    in-tree once, with nvcc for sm_100a, before the tests load it."""
+    from calibrated_block_sparse_calib_b200 import build
+    if not os.path.exists(build.LIB):
+        build.build()
+
+
 def to64(t):
     """bf16/fp32 torch tensor or array -> float64 numpy (exact upcast)."""
     try:
