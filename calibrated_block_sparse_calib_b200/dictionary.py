@@ -23,7 +23,8 @@ The method calibrates offline and keeps, per timestep, layer and head, a static 
       }
 
 Repeat heads use anchor-space query blocks: their rows past the anchor sequence are empty.
-Every conversion runs in the library's kernels; this module only moves buffers and bytes.
+Every conversion runs in the library's kernels; this module moves buffers and bytes, and
+checks a file's header and run structure on the host before any of it reaches the device.
 """
 from __future__ import annotations
 
@@ -37,6 +38,22 @@ import torch
 from . import ops
 
 MAGIC = b"CBSDICT1"
+
+
+def _check_runs(key, iv_ptr: np.ndarray, starts: np.ndarray, lens: np.ndarray, n: int, nk: int):
+    """A slice read from a file must describe a valid skip list before it is expanded on
+    the device: offsets from 0 to n, non-decreasing; every run non-empty and inside
+    [0, nk); runs of a row ascending and disjoint (each starts past the previous one's end)."""
+    ptr = iv_ptr.astype(np.int64)
+    if ptr[0] != 0 or ptr[-1] != n or np.any(np.diff(ptr) < 0):
+        raise ValueError(f"slice {key}: run offsets must rise from 0 to {n}")
+    st, ln = starts.astype(np.int64), lens.astype(np.int64)
+    if n and (st.min() < 0 or ln.min() < 1 or (st + ln).max() > nk):
+        raise ValueError(f"slice {key}: a run is empty or outside the {nk} key blocks")
+    row = np.repeat(np.arange(ptr.size - 1), np.diff(ptr))
+    same = row[1:] == row[:-1]
+    if np.any(st[1:][same] < (st + ln)[:-1][same]):
+        raise ValueError(f"slice {key}: runs of a row overlap or are out of order")
 
 
 @dataclass
@@ -121,11 +138,15 @@ class MaskDictionary:
         if buf[:8] != MAGIC:
             raise ValueError("not a calibrated mask dictionary (bad magic)")
         T, L, H, nq, nk, block, stride, n_slices = struct.unpack_from("<8i", buf, 8)
+        if min(T, L, H, nq, nk, stride) < 1 or block not in (64, 128) or nk > 32767 or n_slices < 0:
+            raise ValueError(f"bad header {(T, L, H, nq, nk, block, stride, n_slices)}")
         d = cls(T, L, H, nq, nk, block, stride)
         off = 40
         for _ in range(n_slices):
             t, l, n = struct.unpack_from("<3i", buf, off)
             off += 12
+            if not 0 <= n <= H * nq * nk:
+                raise ValueError(f"slice {(t, l)}: {n} runs for {H * nq} rows of {nk} blocks")
             rep = tuple(bool(x) for x in np.frombuffer(buf, np.uint8, H, off))
             off += H + (-H % 4)
             iv_ptr = np.frombuffer(buf, "<i4", H * nq + 1, off).astype(np.int32)
@@ -133,8 +154,7 @@ class MaskDictionary:
             starts = np.frombuffer(buf, "<i2", n, off).astype(np.int16)
             lens = np.frombuffer(buf, "<i2", n, off + 2 * n).astype(np.int16)
             off += 4 * n + (-(4 * n) % 4)
-            if int(iv_ptr[-1]) != n:
-                raise ValueError(f"slice {(t, l)}: run offsets end at {int(iv_ptr[-1])}, expected {n}")
+            _check_runs((t, l), iv_ptr, starts, lens, n, nk)
             d._check_key(t, l)
             d.slices[(t, l)] = _Slice(torch.from_numpy(iv_ptr.copy()).to(device),
                                       torch.from_numpy(starts.copy()).to(device),

@@ -1,6 +1,8 @@
 """The mask dictionary's file format, round-tripped on the CPU with oracle-made slices
 (no kernel involved): every array, flag and header field survives, and damaged files are
 rejected."""
+import struct
+
 import numpy as np
 import pytest
 import torch
@@ -61,3 +63,43 @@ def test_keys_outside_the_grid_are_rejected():
     d = MaskDictionary(2, 2, 1, 1, 1, 64)
     with pytest.raises(KeyError):
         d._check_key(2, 0)
+
+
+def _one_slice_bytes(iv_ptr, starts, lens, H=1, nq=2, nk=8, block=64):
+    d = MaskDictionary(1, 1, H, nq, nk, block)
+    d.slices[(0, 0)] = _Slice(torch.tensor(iv_ptr, dtype=torch.int32), torch.tensor(starts, dtype=torch.int16),
+                              torch.tensor(lens, dtype=torch.int16), (False,) * H)
+    return d.to_bytes()
+
+
+def test_run_structure_is_checked_before_upload():
+    """A slice whose runs could not have come from a mask is refused on the host: the
+    device expansion would otherwise write past the skip list it sizes from the runs."""
+    good = _one_slice_bytes([0, 2, 3], [0, 4, 1], [2, 3, 7])
+    e = MaskDictionary.from_bytes(good, device="cpu")
+    assert e.slices[(0, 0)].lens.tolist() == [2, 3, 7]
+    bad_cases = {
+        "empty run": ([0, 2, 3], [0, 4, 1], [2, 0, 7]),
+        "run past nk": ([0, 2, 3], [0, 4, 1], [2, 5, 7]),
+        "negative start": ([0, 2, 3], [0, 4, -1], [2, 3, 7]),
+        "overlapping runs": ([0, 2, 3], [0, 1, 1], [2, 3, 7]),
+        "runs out of order": ([0, 2, 3], [4, 0, 1], [3, 2, 7]),
+        "offsets not from 0": ([1, 2, 3], [0, 4, 1], [2, 3, 7]),
+        "offsets decreasing": ([0, 4, 3], [0, 4, 1], [2, 3, 7]),
+    }
+    for name, (ip, st, ln) in bad_cases.items():
+        with pytest.raises(ValueError):
+            MaskDictionary.from_bytes(_one_slice_bytes(ip, st, ln), device="cpu")
+
+
+def test_bad_headers_are_refused():
+    buf = bytearray(_one_slice_bytes([0, 1, 1], [0], [1]))
+    for field, value in ((5, 96), (4, 0), (7, -1)):     # block 96, nk 0, n_slices -1
+        b = bytearray(buf)
+        struct.pack_into("<i", b, 8 + 4 * field, value)
+        with pytest.raises(ValueError):
+            MaskDictionary.from_bytes(bytes(b), device="cpu")
+    b = bytearray(buf)
+    struct.pack_into("<i", b, 40 + 8, -5)                # a negative run count
+    with pytest.raises(ValueError):
+        MaskDictionary.from_bytes(bytes(b), device="cpu")
