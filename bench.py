@@ -179,6 +179,100 @@ def _time_graph(fn, calls, torch, replays=5):
     return ms
 
 
+def _time_flushed(fn, iters, torch, flush):
+    """Median device time of fn() over `iters` launches, each after a write of `flush` (a
+    buffer larger than L2), so every launch reads its inputs from HBM."""
+    st = torch.cuda.current_stream()
+    fn()
+    ts = []
+    for _ in range(iters):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(st)
+        fn()
+        e1.record(st)
+        e1.synchronize()
+        ts.append(e0.elapsed_time(e1))
+    return statistics.median(ts)
+
+
+def select_leg(energy, taus, torch, ops, flush, peaks, iters=10):
+    """One batched selection launch over energy [nb, H, nq, nk] (per-entry masks written),
+    timed with L2 flushed before each launch.  Bytes: energies read + masks written."""
+    nb = energy.shape[0]
+    msk = torch.empty(energy.shape, dtype=torch.uint8, device=energy.device)
+    ms = _time_flushed(lambda: ops.select_mask_batched(energy, taus, out=msk), iters, torch, flush)
+    nbytes = energy.numel() * (4 + 1)
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    return {"shape": list(energy.shape), "entries": nb, "ms": ms, "bytes": nbytes, "gbs": gbs,
+            "frac_hbm": gbs / peaks["hbm_gbs"], "kept_density": float(msk.float().mean().item()),
+            "kernel": f"select_mask_kernel<{_mpl(energy.shape[-1])}>"}
+
+
+def _mpl(nk):
+    for m, cap in ((2, 64), (4, 128), (8, 256), (16, 512), (20, 640)):
+        if nk <= cap:
+            return m
+    return 32
+
+
+def config_leg(name, wl, timestep, dev, torch, ops, synth, peaks, steps=20, dense_iters=3, flush=None,
+               with_select=False):
+    """Attention on one more workload shape, each number with its own clock record: kept-only
+    and dense-equivalent TFLOPS, fraction of the bf16 peak, and the speedup over this build's
+    dense kernel; optionally the selection pass on that workload's energies."""
+    s = wl.shape
+    B, D, N, H = s.block, s.D, s.N, s.H
+    q, k, v = synth.make_qkv(wl, device=dev)
+    mask_np = synth.make_head_masks(wl, timestep=timestep)
+    bl = ops.BlockList.from_mask(torch.from_numpy(mask_np).to(dev), B)
+    rep = [h in wl.repeat_heads for h in range(H)]
+    stride = wl.repeat_stride
+    n_anchor = ops.anchor_count(s.F, s.Hl, s.Wl, s.n_text, stride) if any(rep) else None
+    out = torch.empty_like(q)
+    if any(rep):
+        call = lambda: ops.sparse_attn_fwd_repeat(q, k, v, bl, rep, s.F, s.Hl, s.Wl, s.n_text, stride, out=out)
+    else:
+        call = lambda: ops.sparse_attn_fwd(q, k, v, bl, out=out)
+    fk = kept_flops(mask_np, N, D, B, tuple(h for h in range(H) if rep[h]), n_anchor)
+    fd = 4.0 * N * N * D * H
+    gpu_id = _gpu_id(torch, dev)
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize()
+    with ClockSampler(gpu_id) as clk:
+        ms = _time_calls(call, steps, 0, torch)
+    ops.device_check()
+    res = {"workload": name, "H": H, "N": N, "D": D, "block": B, "timestep": timestep, "repeat_heads": sum(rep),
+           "kept_fraction_of_dense": round(fk / fd, 4), "ms": ms, "kept_tflops": fk / (ms * 1e-3) / 1e12,
+           "dense_equiv_tflops": fd / (ms * 1e-3) / 1e12,
+           "frac_of_bf16_peak": fk / (ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
+           "frac_of_sustained": fk / (ms * 1e-3) / 1e12 / peaks["bf16_tflops_sustained"], "clocks": clk.summary()}
+    c = res["clocks"]
+    if c.get("sm_mhz") and c.get("sm_max_mhz"):
+        res["kept_tflops_at_max_clock"] = res["kept_tflops"] * c["sm_max_mhz"] / c["sm_mhz"]
+    if dense_iters:
+        full = torch.ones((H, s.nblk, s.nblk), dtype=torch.uint8, device=dev)
+        bl_dense = ops.BlockList.from_mask(full, B)
+        ms_dense = _time_calls(lambda: ops.sparse_attn_fwd(q, k, v, bl_dense, out=out), dense_iters, 1, torch)
+        res["dense_kernel"] = {"ms": ms_dense, "tflops": fd / (ms_dense * 1e-3) / 1e12}
+        res["speedup_vs_dense"] = ms_dense / ms
+        del bl_dense, full
+    if with_select:
+        E = ops.block_energy(q, k, B)
+        res["select"] = select_leg(E.unsqueeze(0), [0.95], torch, ops, flush, peaks)
+        del E
+    ops.device_check()
+    del q, k, v, out
+    torch.cuda.empty_cache()
+    return res
+
+
+def _gpu_id(torch, dev):
+    gpu_uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    return gpu_uuid if gpu_uuid.startswith("GPU-") else f"GPU-{gpu_uuid}"
+
+
 def cpu_baseline(wl, q, k, v, mask, budget_s: float = 12.0):
     """The float64 oracle on a bounded sample: whole query blocks of head 0 (kept keys only
     enter the softmax), as many as fit in ~budget_s.  Returns kept-only TFLOPS."""
@@ -260,39 +354,34 @@ def run_calibration_sweep(dev, torch, ops, synth):
     """Offline calibration over the sweep workload (12 heads x 32760 tokens, B=128): for each of
     8 timesteps (positional scale 1 + t/8) and 4 seeded inputs, the fused LSE + energy pass, then
     the minimal tau-selection for tau in {0.9, 0.95, 0.99} in two aggregation modes -- per-input
-    masks with the cross-input vote (rho = 1/2), and one selection on the energies summed over
-    the inputs (the kernel's accumulate flag).  Reports times, rates and the kept densities."""
+    masks with the cross-input vote (rho = 1/2; one batched launch over a timestep's 4 inputs
+    accumulates the vote counts), and one selection on the energies averaged over the inputs
+    (the kernel's accumulate flag, then the energy mean).  One more batched launch selects all
+    32 (input, timestep) entries at tau(t).  Reports times, rates and the kept densities."""
     wl = synth.WORKLOADS["sweep"]
     s = wl.shape
     B, N, H, nb = s.block, s.N, s.H, s.nblk
     n_in, taus, T = wl.extra["n_calib"], wl.extra["taus"], wl.timesteps
     st = torch.cuda.current_stream()
     ev = lambda: torch.cuda.Event(enable_timing=True)
-    E = torch.empty((H, nb, nb), dtype=torch.float32, device=dev)
-    Esum = torch.empty_like(E)
+    peaks = _peaks()
+    E_all = torch.empty((T * n_in, H, nb, nb), dtype=torch.float32, device=dev)
+    Esum = torch.empty((H, nb, nb), dtype=torch.float32, device=dev)
     msk = torch.empty((H, nb, nb), dtype=torch.uint8, device=dev)
     counts = torch.empty((H, nb, nb), dtype=torch.int32, device=dev)
-    dens = {"vote": {str(t_): [] for t_ in taus}, "energy_sum": {str(t_): [] for t_ in taus}}
+    dens = {"vote": {str(t_): [] for t_ in taus}, "energy_mean": {str(t_): [] for t_ in taus}}
     e_ms, a_ms, sel_ms = [], [], []
     t_start = time.perf_counter()
     for t in range(T):
         qk = [synth.make_qkv(wl, input_idx=d, device=dev, pos_scale=1.0 + 0.125 * t)[:2] for d in range(n_in)]
-        ops.block_energy(qk[0][0], qk[0][1], B, out=E)        # warm-up
-        for tau in taus:
-            counts.zero_()
-            for d, (q, k) in enumerate(qk):
-                e0, e1, e2 = ev(), ev(), ev()
-                e0.record(st)
-                ops.block_energy(q, k, B, out=E)
-                e1.record(st)
-                ops.select_mask(E, tau, out=msk, count_accum=counts)
-                e2.record(st)
-                torch.cuda.synchronize()
-                if tau == taus[0]:
-                    e_ms.append(e0.elapsed_time(e1))
-                sel_ms.append(e1.elapsed_time(e2))
-            vote = ops.aggregate_masks(counts, n_in, (1, 2))
-            dens["vote"][str(tau)].append(float(vote.float().mean().item()))
+        ops.block_energy(qk[0][0], qk[0][1], B, out=Esum)        # warm-up
+        for d, (q, k) in enumerate(qk):
+            e0, e1 = ev(), ev()
+            e0.record(st)
+            ops.block_energy(q, k, B, out=E_all[t * n_in + d])
+            e1.record(st)
+            torch.cuda.synchronize()
+            e_ms.append(e0.elapsed_time(e1))
         for d, (q, k) in enumerate(qk):
             e0, e1 = ev(), ev()
             e0.record(st)
@@ -300,24 +389,40 @@ def run_calibration_sweep(dev, torch, ops, synth):
             e1.record(st)
             torch.cuda.synchronize()
             a_ms.append(e0.elapsed_time(e1))
+        ops.energy_mean(Esum, n_in, out=Esum)
         for tau in taus:
-            dens["energy_sum"][str(tau)].append(float(ops.select_mask(Esum, tau, out=msk).float().mean().item()))
+            dens["energy_mean"][str(tau)].append(float(ops.select_mask(Esum, tau, out=msk).float().mean().item()))
+        for tau in taus:
+            counts.zero_()
+            e0, e1 = ev(), ev()
+            e0.record(st)
+            ops.select_mask_batched(E_all[t * n_in:(t + 1) * n_in], [tau] * n_in, count_accum=counts,
+                                    write_masks=False)
+            e1.record(st)
+            vote = ops.aggregate_masks(counts, n_in, (1, 2))
+            torch.cuda.synchronize()
+            sel_ms.append(e0.elapsed_time(e1))
+            dens["vote"][str(tau)].append(float(vote.float().mean().item()))
         del qk
+    tau_of = lambda t: 0.99 if t < T // 3 else (0.95 if t < 2 * T // 3 else 0.9)
+    flush = torch.empty(256 * 2**20, dtype=torch.uint8, device=dev)
+    sel_all = select_leg(E_all, [tau_of(t) for t in range(T) for _ in range(n_in)], torch, ops, flush, peaks)
+    del E_all, flush
     # the dictionary of the sweep: one slice per timestep with a stricter tau early on
     # (tau(t) = 0.99, 0.95, 0.9 over the three thirds of the schedule), repetition
     # detection at gamma = 0.9 and stride 4, built by the calibration driver, saved, reloaded
     from calibrated_block_sparse_calib_b200.calibrate import calibrate_slice
     from calibrated_block_sparse_calib_b200.dictionary import MaskDictionary
     import tempfile
-    dct = MaskDictionary(T, 1, H, nb, nb, B, stride=4)
+    dct = MaskDictionary(T, 1, H, nb, nb, B, stride=4, rho=(1, 2), mode="vote", n_inputs=n_in, gamma=0.9)
     members = torch.from_numpy(synth.sample_video_tokens(s, 512, seed=3)).to(dev)
     t_d = time.perf_counter()
     flags = []
     for t in range(T):
-        tau_t = 0.99 if t < T // 3 else (0.95 if t < 2 * T // 3 else 0.9)
+        tau_t = tau_of(t)
         qk = [synth.make_qkv(wl, input_idx=d, device=dev, pos_scale=1.0 + 0.125 * t)[:2] for d in range(n_in)]
         mask_t, rep_t, _ = calibrate_slice(qk, s.F, s.Hl, s.Wl, 0, B, tau_t, (1, 2), "vote", 0.9, 4, members)
-        dct.put_mask(t, 0, mask_t, rep_t)
+        dct.put_mask(t, 0, mask_t, rep_t, tau=tau_t)
         flags.append(sum(rep_t))
         del qk
     torch.cuda.synchronize()
@@ -331,7 +436,7 @@ def run_calibration_sweep(dev, torch, ops, synth):
     ops.device_check()
     em = statistics.median(e_ms)
     sm_ = statistics.median(sel_ms)
-    sel_bytes = H * nb * nb * (4 + 1 + 4 + 4)     # energies in, mask out, vote counts read + written
+    sel_bytes = n_in * H * nb * nb * 4 + H * nb * nb * 8   # 4 inputs' energies in, vote counts read + written
     exps = 2.0 * N * N * H / (em * 1e-3)
     peak = MUFU_EX2_PER_CLK_SM * B200_SMS * 1965.0e6
     print(json.dumps({
@@ -340,7 +445,8 @@ def run_calibration_sweep(dev, torch, ops, synth):
         "energy_ms_median": em, "energy_exp2_per_s": exps, "energy_frac_of_mufu_at_1965mhz": exps / peak,
         "energy_tflops_qk": 2 * 2.0 * N * N * s.D * H / (em * 1e-3) / 1e12,
         "energy_accumulate_ms_median": statistics.median(a_ms),
-        "select_ms_median": sm_, "select_gbs": sel_bytes / (sm_ * 1e-3) / 1e9,
+        "select_vote_launch_ms_median": sm_, "select_vote_launch_gbs": sel_bytes / (sm_ * 1e-3) / 1e9,
+        "select_all_entries": sel_all,
         "kept_density": dens,
         "dictionary": {"slices": T, "tau_schedule": [0.99 if t < T // 3 else (0.95 if t < 2 * T // 3 else 0.9)
                                                      for t in range(T)],
@@ -358,13 +464,14 @@ def main():
     ap.add_argument("--timestep", type=int, default=0, help="timestep of the mask schedule (mochi1)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--no-extras", action="store_true", help="skip dense / e2e / calibration legs")
+    ap.add_argument("--no-extras", action="store_true", help="skip dense / e2e / calibration / other-config legs")
+    ap.add_argument("--no-configs", action="store_true", help="skip the Wan-14B / Mochi-1 legs")
     ap.add_argument("--energy-only", action="store_true",
                     help="time only the fused LSE + block-energy pass (calibration) and print its own line")
     ap.add_argument("--heads", type=int, default=None, help="with --energy-only: the first H heads only")
     ap.add_argument("--calibration-sweep", action="store_true",
                     help="the calibration sweep: energies + selection over 4 inputs x 8 timesteps x 3 taus, "
-                         "cross-input vote and energy-sum modes; prints its own line")
+                         "cross-input vote and energy-mean modes; prints its own line")
     ap.add_argument("--ref-seconds", type=float, default=60.0,
                     help="--impl reference: total seconds of oracle work over the timed steps")
     args = ap.parse_args()
@@ -503,6 +610,14 @@ def main():
             msk = torch.empty(energy.shape, dtype=torch.uint8, device=dev)
             ms_sel = _time_graph(lambda: ops.select_mask(energy, 0.95, out=msk), 20, torch)
             sel_bytes = energy.numel() * 4 + msk.numel()
+            # the calibration sweep's shape: 4 inputs x 8 timesteps of these energies in one
+            # launch (each entry its own copy in HBM, tau(t) per timestep), L2 flushed before
+            # every launch
+            flush = torch.empty(256 * 2**20, dtype=torch.uint8, device=dev)
+            batch = energy.unsqueeze(0).repeat(32, 1, 1, 1)
+            taus32 = [0.99 if t < 3 else (0.95 if t < 6 else 0.9) for t in range(8) for _ in range(4)]
+            sel_batched = select_leg(batch, taus32, torch, ops, flush, peaks)
+            del batch
             # LSE reuse: a dense forward that emits the row LSE (calibration runs the dense
             # model anyway), then the energy pass with that LSE runs a single pass
             lse_buf = torch.empty((H, N), dtype=torch.float32, device=dev)
@@ -523,7 +638,8 @@ def main():
                                     "peak_source": "16 MUFU ex2 per clock per SM x 148 SMs x max SM clock"},
                 "select_ms": ms_sel, "select_gbs": sel_bytes / (ms_sel * 1e-3) / 1e9,
                 "select_frac_hbm": sel_bytes / (ms_sel * 1e-3) / 1e9 / peaks["hbm_gbs"],
-                "tau": 0.95, "selected_density": float(msk.float().mean().item())}
+                "tau": 0.95, "selected_density": float(msk.float().mean().item()),
+                "select_batched_32": sel_batched}
             # spatial-repetition detection: cosine of 1024 sampled tokens' attention rows
             # against their stride-4 anchors, two passes over K, then the per-head decision
             mem = torch.from_numpy(synth.sample_video_tokens(s, 1024, seed=1)).to(dev)
@@ -551,6 +667,18 @@ def main():
                 "encode_ms": ms_enc}
             ops.device_check()
 
+    # the other model-shaped workloads, each under its own clock record (replica 0 of a
+    # multi-GPU run measures them; the others wait at the final barrier)
+    if not args.no_extras and not args.no_configs and wl.name == "wan13b" and rank == 0:
+        flush = torch.empty(256 * 2**20, dtype=torch.uint8, device=dev)
+        extras["configs"] = {
+            "wan14b720p": config_leg("wan14b720p", synth.WORKLOADS["wan14b720p"], 0, dev, torch, ops, synth, peaks,
+                                     steps=10, dense_iters=2, flush=flush, with_select=True),
+            "mochi1_t0": config_leg("mochi1", synth.WORKLOADS["mochi1"], 0, dev, torch, ops, synth, peaks,
+                                    steps=20, dense_iters=2),
+            "mochi1_t7": config_leg("mochi1", synth.WORKLOADS["mochi1"], 7, dev, torch, ops, synth, peaks,
+                                    steps=20, dense_iters=0),
+        }
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",

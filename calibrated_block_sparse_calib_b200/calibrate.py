@@ -9,9 +9,11 @@ For every head of the slice ([zh] §2.2A, [de] §2A.1-§2A.5, [fr] §2.B of the 
    per-head decision mean > gamma (calib_repeat_flags);
 2. block energies per input, over all query rows (calib_block_energy), and over the anchor
    rows for the flagged heads (their masks live in anchor query-block space);
-3. per-input minimal tau-selection with vote counts (calib_select_mask) and the
-   cross-input vote (calib_aggregate_masks), or selection on the energies summed over the
-   inputs (the energy kernel's accumulate flag);
+3. either the pages' vote -- per-input minimal tau-selection of all inputs in one batched
+   launch that accumulates the vote counts (calib_select_mask_batched), then the
+   cross-input vote (calib_aggregate_masks) -- or the energy mean: energies summed over the
+   inputs (the energy kernel's accumulate flag), divided by the number of inputs
+   (calib_energy_mean) and selected once (calib_select_mask);
 4. the slice mask: a flagged head takes its anchor-space rows (the rest of its rows stay
    empty), the others their full-space rows.
 
@@ -35,7 +37,8 @@ def calibrate_slice(inputs: List[Tuple[torch.Tensor, torch.Tensor]], F: int, Hl:
     """Returns (mask uint8 [H, nq, nk], repeat bool list [H], details dict).
 
     inputs     : per calibration input, (q, k) bf16 [H, N, D] on the device.
-    mode       : "vote" (per-input masks, strict vote above rho) or "energy_sum".
+    mode       : "vote" (per-input masks, strict vote above rho) or "energy_mean" (block
+                 energies averaged over the inputs, then one selection).
     gamma      : repetition threshold, or None to skip detection (no head repeats).
     members    : int32 [n] sampled video tokens for detection (required with gamma).
     force_keep : uint8 [H, nq, nk] blocks always kept (e.g. text rows / columns).
@@ -43,8 +46,8 @@ def calibrate_slice(inputs: List[Tuple[torch.Tensor, torch.Tensor]], F: int, Hl:
                  with force_keep when a head is flagged (text rows sit at the end of the
                  compacted anchor sequence, so the full-space rows do not carry over).
     """
-    if mode not in ("vote", "energy_sum"):
-        raise ValueError("mode must be 'vote' or 'energy_sum'")
+    if mode not in ("vote", "energy_mean"):
+        raise ValueError("mode must be 'vote' or 'energy_mean'")
     q0, k0 = inputs[0]
     H, N, D = q0.shape
     dev = q0.device
@@ -65,17 +68,19 @@ def calibrate_slice(inputs: List[Tuple[torch.Tensor, torch.Tensor]], F: int, Hl:
     # 2-3. energies and selection, full space and (if needed) anchor space
     def select_space(q_rows=None, nq_space=nq, force=None):
         shape = (H, nq_space, nk)
+        n_in = len(inputs)
         if mode == "vote":
+            energies = torch.empty((n_in,) + shape, dtype=torch.float32, device=dev)
+            for d, (q, k) in enumerate(inputs):
+                ops.block_energy(q, k, block, q_rows=q_rows, out=energies[d])
             counts = torch.zeros(shape, dtype=torch.int32, device=dev)
-            msk = torch.empty(shape, dtype=torch.uint8, device=dev)
-            for q, k in inputs:
-                e = ops.block_energy(q, k, block, q_rows=q_rows)
-                ops.select_mask(e, tau, force_keep=force, out=msk, count_accum=counts)
-            return ops.aggregate_masks(counts, len(inputs), rho)
+            ops.select_mask_batched(energies, [tau] * n_in, force_keep=force, count_accum=counts,
+                                    write_masks=False)
+            return ops.aggregate_masks(counts, n_in, rho)
         esum = None
-        for i, (q, k) in enumerate(inputs):
-            esum = ops.block_energy(q, k, block, q_rows=q_rows, out=esum, accumulate=i > 0)
-        return ops.select_mask(esum, tau, force_keep=force)
+        for d, (q, k) in enumerate(inputs):
+            esum = ops.block_energy(q, k, block, q_rows=q_rows, out=esum, accumulate=d > 0)
+        return ops.select_mask(ops.energy_mean(esum, n_in, out=esum), tau, force_keep=force)
 
     mask = select_space(force=force_keep)
     if any(repeat):

@@ -5,6 +5,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <type_traits>
@@ -320,8 +321,7 @@ calib_status calib_device_check(void* stream) {
     if (cudaMemcpyFromSymbol(&v, calib::g_status, sizeof(v)) != cudaSuccess) return CALIB_ERR_CUDA;
     if (v && cudaMemcpyToSymbol(calib::g_status, &zero, sizeof(zero)) != cudaSuccess) return CALIB_ERR_CUDA;
     if (v & calib::STATUS_TIMEOUT) return CALIB_ERR_TIMEOUT;
-    if (v & calib::STATUS_SMEM_ALIGN) return CALIB_ERR_CUDA;
-    if (v & calib::STATUS_BAD_ENERGY) return CALIB_ERR_INVALID;
+    if (v & (calib::STATUS_BAD_ENERGY | calib::STATUS_BAD_LIST)) return CALIB_ERR_INVALID;
     return CALIB_OK;
 }
 
@@ -357,18 +357,39 @@ calib_status calib_block_energy(const void* q, const void* k, const float* lse, 
     return block == 128 ? launch_energy<64, 128>(tk, p, grid, st) : launch_energy<64, 64>(tk, p, grid, st);
 }
 
-calib_status calib_select_mask(const float* energy, int H, int nq, int nk, double tau, const uint8_t* force_keep,
-                               uint8_t* mask_out, int32_t* count_accum, void* stream) {
-    if (!energy || !mask_out) return CALIB_ERR_INVALID;
-    if (H < 1 || nq < 1 || nk < 1 || !(tau > 0.0) || !(tau <= 1.0)) return CALIB_ERR_INVALID;
+calib_status calib_select_mask_batched(const float* energy, int nb, int H, int nq, int nk, const double* tau,
+                                       const uint8_t* force_keep, uint8_t* mask_out, int32_t* count_accum,
+                                       void* stream) {
+    if (!energy || !tau || (!mask_out && !count_accum)) return CALIB_ERR_INVALID;
+    if (nb < 1 || nb > calib::kSelMaxBatch || H < 1 || nq < 1 || nk < 1) return CALIB_ERR_INVALID;
     if (nk > 32 * calib::kSelMaxPerLane) return CALIB_ERR_UNSUPPORTED;
-    if (static_cast<long long>(H) * nq * nk > (1ll << 31) - 1) return CALIB_ERR_INVALID;
+    if ((reinterpret_cast<uintptr_t>(energy) & 3u) || (reinterpret_cast<uintptr_t>(count_accum) & 3u))
+        return CALIB_ERR_INVALID;
+    if (static_cast<long long>(nb) * H * nq * nk > (1ll << 31) - 1) return CALIB_ERR_INVALID;
+    for (int b = 0; b < nb; ++b)
+        if (!(tau[b] > 0.0) || !(tau[b] <= 1.0)) return CALIB_ERR_INVALID;
     if (calib_status s = check_device()) return s;
-    const int rows = H * nq;
+    calib::SelectParams p{};
+    p.energy = energy;
+    p.force = force_keep;
+    p.mask_out = mask_out;
+    p.count_accum = count_accum;
+    p.nb = nb; p.rows = H * nq; p.nq = nq; p.nk = nk;
+    for (int b = 0; b < nb; ++b) p.tau[b] = tau[b];
+    // one warp per (row, chunk of entries): enough warps to fill every SM a few times over,
+    // and each warp walks its chunk of entries so that vote counts accumulate in registers
+    const long long target = 148ll * 48;
+    int n_chunks = static_cast<int>(std::min<long long>(nb, std::max<long long>(1, (target + p.rows - 1) / p.rows)));
+    p.chunk = (nb + n_chunks - 1) / n_chunks;
+    p.n_chunks = (nb + p.chunk - 1) / p.chunk;
+    p.vec = ((nk & 3) == 0 && (reinterpret_cast<uintptr_t>(energy) & 15u) == 0 &&
+             (!mask_out || (reinterpret_cast<uintptr_t>(mask_out) & 3u) == 0)) ? 1 : 0;
+    const long long warps = static_cast<long long>(p.rows) * p.n_chunks;
+    const int grid = static_cast<int>((warps + calib::kSelWarps - 1) / calib::kSelWarps);
+    cudaStream_t st = as_stream(stream);
     // energies per lane: the smallest instantiated count covering the row
     auto launch = [&](auto mpl) {
-        calib::select_mask_kernel<decltype(mpl)::value><<<rows_grid(rows), 128, 0, as_stream(stream)>>>(
-            energy, rows, nq, nk, tau, force_keep, mask_out, count_accum);
+        calib::select_mask_kernel<decltype(mpl)::value><<<grid, calib::kSelWarps * 32, 0, st>>>(p);
     };
     if (nk <= 64) launch(std::integral_constant<int, 2>{});
     else if (nk <= 128) launch(std::integral_constant<int, 4>{});
@@ -376,6 +397,25 @@ calib_status calib_select_mask(const float* energy, int H, int nq, int nk, doubl
     else if (nk <= 512) launch(std::integral_constant<int, 16>{});
     else if (nk <= 640) launch(std::integral_constant<int, 20>{});
     else launch(std::integral_constant<int, 32>{});
+    return launch_status();
+}
+
+calib_status calib_select_mask(const float* energy, int H, int nq, int nk, double tau, const uint8_t* force_keep,
+                               uint8_t* mask_out, int32_t* count_accum, void* stream) {
+    if (!mask_out) return CALIB_ERR_INVALID;
+    return calib_select_mask_batched(energy, 1, H, nq, nk, &tau, force_keep, mask_out, count_accum, stream);
+}
+
+calib_status calib_energy_mean(const float* energy_sum, int64_t count, int n_inputs, float* mean_out,
+                               void* stream) {
+    if (!energy_sum || !mean_out || count < 1 || n_inputs < 1 || n_inputs > (1 << 24)) return CALIB_ERR_INVALID;
+    if ((reinterpret_cast<uintptr_t>(energy_sum) & 3u) || (reinterpret_cast<uintptr_t>(mean_out) & 3u))
+        return CALIB_ERR_INVALID;
+    if (calib_status s = check_device()) return s;
+    const long long want = (count / 4 + 255) / 256;
+    const int grid = static_cast<int>(std::max<long long>(1, std::min<long long>(want, 148ll * 8)));
+    calib::energy_mean_kernel<<<grid, 256, 0, as_stream(stream)>>>(energy_sum, count, static_cast<float>(n_inputs),
+                                                                   mean_out);
     return launch_status();
 }
 
@@ -546,6 +586,30 @@ calib_status sparse_attn_fwd_repeat(const void* q, const void* k, const void* v,
     int N = 0;
     if (calib_status s = repeat_geometry(H, F, Hl, Wl, n_text, stride, head_repeat, bits, &N)) return s;
     return attn_common(q, k, v, o, lse_opt, H, N, D, scale, list, bits, F, Hl, Wl, n_text, stride, flags, stream);
+}
+
+calib_status calib_validate_block_list_host(int H, int nq, int nk, const int32_t* row_ptr, const int16_t* col_idx,
+                                            int64_t col_capacity, const int32_t* work, int n_work) {
+    if (H < 1 || nq < 1 || nk < 1 || nk > 32767 || !row_ptr || col_capacity < 0) return CALIB_ERR_INVALID;
+    const long long rows = static_cast<long long>(H) * nq;
+    if (rows > (1ll << 31) - 2 || row_ptr[0] != 0) return CALIB_ERR_INVALID;
+    for (long long r = 0; r < rows; ++r) {
+        const long long b = row_ptr[r], e = row_ptr[r + 1];
+        if (e < b || e - b > nk || e > col_capacity) return CALIB_ERR_INVALID;
+        if (e > b && !col_idx) return CALIB_ERR_INVALID;
+        for (long long x = b; x < e; ++x) {
+            const int j = col_idx[x];
+            if (j < 0 || j >= nk || (x > b && j <= col_idx[x - 1])) return CALIB_ERR_INVALID;
+        }
+    }
+    if (work) {
+        if (n_work < 0) return CALIB_ERR_INVALID;
+        for (int w = 0; w < n_work; ++w) {
+            const int32_t item = work[w];
+            if (item < 0 || (item >> 16) >= H || (item & 0xFFFF) >= nq) return CALIB_ERR_INVALID;
+        }
+    }
+    return CALIB_OK;
 }
 
 calib_status calib_selftest_wait_timeout(uint32_t timeout_us, void* stream) {

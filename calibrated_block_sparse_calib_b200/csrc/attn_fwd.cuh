@@ -149,12 +149,22 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         h = blockIdx.x / p.nq;
         i = blockIdx.x - h * p.nq;
     }
+    // A work item or row outside the call is skipped (and reported) before anything depends
+    // on it; the values are the same in every thread, so the whole CTA leaves together.
+    if (h < 0 || h >= p.H || i >= p.nq) {
+        if (threadIdx.x == 0) raise_status(STATUS_BAD_LIST);
+        return;
+    }
     const bool rep = (p.repeat_bits[h >> 5] >> (h & 31)) & 1u;
     const int Nq = rep ? p.n_anchor : p.N;
     if (i >= (rep ? p.nq_anchor : p.nq)) return;  // rows past a repeat head's anchor space
     const int lrow = h * p.nq + i;
     const int kbeg = p.row_ptr[lrow];
     const int nkept = p.row_ptr[lrow + 1] - kbeg;
+    if (kbeg < 0 || nkept < 0 || nkept > p.nk) {
+        if (threadIdx.x == 0) raise_status(STATUS_BAD_LIST);
+        return;
+    }
 
     // ---- setup ------------------------------------------------------------------
     // The first softmax warps fetch their Q rows into registers now, so that the global
@@ -361,7 +371,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         bool ok = true;
         for (int t = 0; t < nkept; ++t) {
             const int j = p.col_idx[kidx(t)];
-            const int valid = min(BLK, p.N - j * BLK) - hf * HC;   // may be <= 0 (ragged tail)
+            // may be <= 0: the ragged tail, or an index outside the key blocks (masked whole)
+            const int valid = (j >= 0 ? min(BLK, p.N - j * BLK) : 0) - hf * HC;
             ok = mbar_wait_warp(bar(L::B_SF), t & 1, ctl);
             if (!ok) break;
             tc_fence_after();

@@ -11,7 +11,11 @@ namespace calib {
 // ------------------------------------------------------------------------------------
 // Device status word (one per device, in this translation unit).
 // ------------------------------------------------------------------------------------
-enum : uint32_t { STATUS_TIMEOUT = 1u, STATUS_BAD_ENERGY = 2u, STATUS_SMEM_ALIGN = 4u };
+// TIMEOUT: a bounded wait gave up.  BAD_ENERGY: selection met a negative or non-finite
+// energy (counted as 0).  BAD_LIST: an attention work item named a head or query block
+// outside the call, or a row whose pointers are negative or decreasing, or keep more
+// than nk blocks; the item was skipped.
+enum : uint32_t { STATUS_TIMEOUT = 1u, STATUS_BAD_ENERGY = 2u, STATUS_BAD_LIST = 4u };
 __device__ uint32_t g_status;
 
 __device__ __forceinline__ void raise_status(uint32_t bits) { atomicOr(&g_status, bits); }

@@ -7,161 +7,329 @@
 namespace calib {
 
 constexpr int kSelMaxPerLane = 32;   // nk <= 32 * 32 = 1024 in selection
+constexpr int kSelMaxBatch = 256;    // energy matrices per selection call
+constexpr int kSelWarps = 4;         // warps per CTA of the selection kernel
+constexpr int kSelCompact = 64;      // largest candidate set moved to shared memory
+
+// Parameters of one batched selection call.  Batch entry b is the energy matrix
+// energy[b] of shape [rows, nk] (rows = H * nq); force_keep and count_accum are shared by
+// every entry.
+struct SelectParams {
+    const float* energy;       // [nb, rows, nk]
+    const uint8_t* force;      // [rows, nk] or null
+    uint8_t* mask_out;         // [nb, rows, nk] or null
+    int32_t* count_accum;      // [rows, nk] or null: += the number of entries keeping (r, j)
+    int nb, rows, nq, nk;
+    int chunk, n_chunks;       // batch entries per warp; warps per row
+    int vec;                   // 1: rows and lane chunks are 16-byte aligned (vector loads)
+    double tau[kSelMaxBatch];
+};
 
 __device__ __forceinline__ uint32_t lanemask_lt() {
     uint32_t m;
     asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
     return m;
 }
-__device__ __forceinline__ uint64_t warp_sum_u64(uint64_t v) {
+__device__ __forceinline__ uint32_t warp_sum_u32(uint32_t v) { return __reduce_add_sync(0xffffffffu, v); }
+__device__ __forceinline__ uint32_t warp_max_u32(uint32_t v) { return __reduce_max_sync(0xffffffffu, v); }
+// Exclusive prefix sum over the lanes of a warp.
+__device__ __forceinline__ uint32_t warp_exclusive_scan(uint32_t v) {
+    const uint32_t lane = lane_id();
+    uint32_t x = v;
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
-    return v;
-}
-__device__ __forceinline__ uint64_t warp_max_u64(uint64_t v) {
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-        const uint64_t o = __shfl_xor_sync(0xffffffffu, v, off);
-        v = o > v ? o : v;
+    for (int off = 1; off < 32; off <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, x, off);
+        if (lane >= static_cast<uint32_t>(off)) x += y;
     }
-    return v;
+    return x - v;
 }
 
 // Exponent p with x < 2^p <= 2x for finite x > 0 (the exponent frexp returns), read from
 // the IEEE-754 binary32 fields.
-__device__ __forceinline__ int float_exponent_p(float x) {
-    const uint32_t bits = __float_as_uint(x);
+__device__ __forceinline__ int float_exponent_p(uint32_t bits) {
     const int E = static_cast<int>((bits >> 23) & 0xFFu);
     if (E != 0) return E - 126;
     const int msb = 31 - __clz(bits & 0x7FFFFFu);   // subnormal: value = mant * 2^-149
     return msb - 148;
 }
 
-// Minimal tau-energy selection, one warp per row, MPL energies per lane (nk <= 32 * MPL).
-// See calib_select_mask in calibatt.h for the rule; the kept set is forced blocks, then
-// every non-forced block with q_j > v, then the first c non-forced blocks (ascending j)
-// with q_j == v, where v is the largest value with F + sum_{q_j >= v} q_j >= T.
+// q = rint(e * 2^shift), ties to even, for e >= 0 given by its binary32 bits x.  The
+// significand m and exponent give e = m * 2^(E' - 150) (E' = max(E, 1)), so q = m * 2^k
+// with k = E' - 150 + shift: a left shift when k >= 0, else a right shift by s = -k with
+// round-half-even on the bits shifted out.  This is the same integer that rounding the
+// (exact) binary64 product e * 2^shift gives.
+__device__ __forceinline__ uint64_t quantize_bits(uint32_t x, int shift) {
+    const uint32_t E = x >> 23;
+    const uint32_t m = E ? ((x & 0x7FFFFFu) | 0x800000u) : (x & 0x7FFFFFu);
+    const int k = static_cast<int>(E ? E : 1u) - 150 + shift;
+    if (k >= 0) return static_cast<uint64_t>(m) << k;
+    const int s = -k;
+    if (s >= 32) return 0;
+    const uint32_t qt = m >> s;
+    const uint32_t rem = m & ((1u << s) - 1u);
+    const uint32_t half = 1u << (s - 1);
+    return qt + ((rem > half || (rem == half && (qt & 1u))) ? 1u : 0u);
+}
+
+// Minimal tau-energy selection, one warp per (row, chunk of batch entries); lane l holds
+// key blocks [l*MPL, (l+1)*MPL) of the row (nk <= 32*MPL).  See calib_select_mask in
+// calibatt.h for the rule.  With q_j the row's integer energies (shift chosen so that the
+// total stays below 2^53), forced total F and threshold T, the kept set is: the forced
+// blocks, every free block with q_j > v, and the first c free blocks (ascending j) with
+// q_j == v, where v is the largest value with F + sum_{free, q_j >= v} q_j >= T.
 //
-// v is found by bisection over the binary32 bit patterns b_j of the energies rather than
-// over the integer values: for e >= 0 the bit pattern is monotone in e and q_j =
-// rint(e_j 2^shift) is monotone in e_j, so with G(u) = F + sum_{free, b_j >= u} q_j the
-// largest u with G(u) >= T is the pattern of an energy whose q is exactly v (G steps only
-// at element patterns, and a step with q = 0 changes nothing).  That takes at most 31
-// steps with 32-bit compares; every sum stays an exact 64-bit integer.
-// (16 and 20 energies per lane: six CTAs per SM, trading a few spilled registers for the
-// occupancy that hides the bisection's shuffle latency; measured 20% faster at nk = 591)
+// Finding v.  For e >= 0 the binary32 bit pattern b is monotone in e, and q is monotone in
+// e, so with G(u) = F + sum_{free, b_j >= u} q_j the largest pattern u* with G(u*) >= T is
+// the pattern of a free energy whose q is exactly v (G changes only where an element with
+// q > 0 drops out).  u* is found in two bisections:
+//   1. over the exponent field: the largest level e with G(e << 23) >= T (at most 8 steps
+//      over all of the row's elements);
+//   2. over the 23 low bits inside that level, where only the elements of that level can
+//      change G; when they are few (<= 64, the usual case: a factor-of-two band of
+//      energies) they are first moved to shared memory, two per lane, so each step
+//      touches two values instead of MPL.
+// Every sum is exact: q_j < 2^(52-c) with c = ceil(log2 nk) is split at bit 32-c into a
+// low part (row total < 2^32) and a high part (row total < 2^30), each reduced over the
+// warp with one 32-bit redux.
 template <int MPL>
-__global__ void __launch_bounds__(128, MPL <= 8 ? 8 : (MPL <= 20 ? 6 : 3))
-select_mask_kernel(const float* __restrict__ energy, int rows, int nq, int nk, double tau,
-                   const uint8_t* __restrict__ force, uint8_t* __restrict__ mask_out,
-                   int32_t* __restrict__ count_accum) {
+__global__ void __launch_bounds__(kSelWarps * 32, MPL <= 8 ? 8 : (MPL <= 16 ? 6 : (MPL <= 20 ? 5 : 3)))
+select_mask_kernel(const __grid_constant__ SelectParams p) {
     static_assert(MPL >= 1 && MPL <= kSelMaxPerLane, "per-lane count");
-    const int row = blockIdx.x * (blockDim.x >> 5) + static_cast<int>(warp_id());
-    if (row >= rows) return;
+    __shared__ uint32_t cand_b[kSelWarps][kSelCompact];
+    __shared__ uint32_t cand_l[kSelWarps][kSelCompact];
+    __shared__ uint32_t cand_h[kSelWarps][kSelCompact];
+    const uint32_t wib = warp_id();
+    const long long gw = static_cast<long long>(blockIdx.x) * kSelWarps + wib;
+    if (gw >= static_cast<long long>(p.rows) * p.n_chunks) return;
+    const int row = static_cast<int>(gw % p.rows);
+    const int ck = static_cast<int>(gw / p.rows);
+    const int bfirst = ck * p.chunk, blast = min(p.nb, bfirst + p.chunk);
     const uint32_t lane = lane_id();
-    const int i = row % nq;
-    const size_t base = static_cast<size_t>(row) * nk;
+    const int nk = p.nk;
+    const int i = row % p.nq;
+    const int j0 = static_cast<int>(lane) * MPL;
+    const size_t rbase = static_cast<size_t>(row) * nk;
+    const int c = nk <= 1 ? 0 : 32 - __clz(nk - 1);
+    const int cs = 32 - c;                                   // split bit of q: 22..32
+    const uint32_t lomask = cs >= 32 ? 0xFFFFFFFFu : ((1u << cs) - 1u);
+    auto join = [&](uint32_t hi_sum, uint32_t lo_sum) -> uint64_t {
+        return (static_cast<uint64_t>(hi_sum) << cs) + lo_sum;
+    };
 
-    float ev[MPL];
-    uint32_t fbits = 0;
-    float emax = 0.f;
-    bool bad = false;
+    uint32_t fbits = 0;                                      // forced blocks of this row
+    if (p.force) {
 #pragma unroll
-    for (int m = 0; m < MPL; ++m) {
-        const int j = static_cast<int>(lane) + 32 * m;
-        float x = 0.f;
-        if (j < nk) {
-            x = energy[base + j];
-            if (!(x >= 0.f) || x == INFINITY) { bad = true; x = 0.f; }
-            if (force && force[base + j]) fbits |= 1u << m;
-        }
-        ev[m] = x;
-        emax = fmaxf(emax, x);
+        for (int m = 0; m < MPL; ++m)
+            if (j0 + m < nk && p.force[rbase + j0 + m]) fbits |= 1u << m;
     }
+    uint32_t cnt[(MPL + 3) / 4];                             // keep counts, one byte per block
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) emax = fmaxf(emax, __shfl_xor_sync(0xffffffffu, emax, off));
-    if (__any_sync(0xffffffffu, bad) && lane == 0) raise_status(STATUS_BAD_ENERGY);
+    for (int w = 0; w < (MPL + 3) / 4; ++w) cnt[w] = 0;
 
-    uint32_t kbits = fbits;
-    if (emax > 0.f) {
-        const int p = float_exponent_p(emax);
-        const int c = nk <= 1 ? 0 : 32 - __clz(nk - 1);
-        const int shift = 52 - p - c;                                   // in [-86, 200]
-        const double two_shift = __longlong_as_double(static_cast<long long>(shift + 1023) << 52);
-        uint64_t q[MPL];
-        uint32_t b[MPL];           // bit pattern of a free energy; 0 for forced and padding
-        uint64_t Ql = 0, Fl = 0;
-        uint32_t bmax = 0;
+    for (int bi = bfirst; bi < blast; ++bi) {
+        const float* E = p.energy + (static_cast<size_t>(bi) * p.rows + row) * nk;
+        uint32_t b[MPL];
+        if constexpr (MPL % 4 == 0) {
+            if (p.vec) {
+#pragma unroll
+                for (int v = 0; v < MPL / 4; ++v) {
+                    float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+                    if (j0 + 4 * v < nk) x = reinterpret_cast<const float4*>(E + j0)[v];
+                    b[4 * v] = __float_as_uint(x.x);
+                    b[4 * v + 1] = __float_as_uint(x.y);
+                    b[4 * v + 2] = __float_as_uint(x.z);
+                    b[4 * v + 3] = __float_as_uint(x.w);
+                }
+            }
+        }
+        if (!(MPL % 4 == 0) || !p.vec) {
+#pragma unroll
+            for (int m = 0; m < MPL; ++m) b[m] = j0 + m < nk ? __float_as_uint(E[j0 + m]) : 0u;
+        }
+        // negative, NaN or infinite energies count as 0 (and are reported); -0 becomes +0
+        bool bad = false;
+        uint32_t xmax = 0;
 #pragma unroll
         for (int m = 0; m < MPL; ++m) {
-            q[m] = __double2ull_rn(__dmul_rn(static_cast<double>(ev[m]), two_shift));   // exact x 2^shift
-            Ql += q[m];
-            const bool fr = (fbits >> m) & 1u;
-            if (fr) Fl += q[m];
-            b[m] = fr ? 0u : __float_as_uint(ev[m]);
-            bmax = b[m] > bmax ? b[m] : bmax;
+            const float x = __uint_as_float(b[m]);
+            if (!(x >= 0.f) || x == INFINITY) bad = true;
+            if (!(x > 0.f) || x == INFINITY) b[m] = 0u;
+            xmax = b[m] > xmax ? b[m] : xmax;
         }
-        const uint64_t Q = warp_sum_u64(Ql);
-        const uint64_t F = warp_sum_u64(Fl);
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) {
-            const uint32_t o = __shfl_xor_sync(0xffffffffu, bmax, off);
-            bmax = o > bmax ? o : bmax;
-        }
-        uint64_t T = __double2ull_rz(ceil(__dmul_rn(tau, __ull2double_rn(Q))));
-        if (T < 1) T = 1;
-        if (F < T) {
-            // G(0) = Q >= T (forced and padding add 0 at u = 0 only through F), G(bmax + 1) = F < T
-            uint32_t lo = 0, hi = bmax + 1;
-            constexpr int NACC = MPL < 4 ? MPL : 4;   // independent partial sums: short add chains
-            while (hi - lo > 1) {
-                const uint32_t mid = lo + ((hi - lo) >> 1);
-                uint64_t acc[NACC];
-#pragma unroll
-                for (int a = 0; a < NACC; ++a) acc[a] = 0;
-#pragma unroll
-                for (int m = 0; m < MPL; ++m)
-                    acc[m % NACC] += b[m] >= mid ? q[m] : 0ull;
-                uint64_t sl = acc[0];
-#pragma unroll
-                for (int a = 1; a < NACC; ++a) sl += acc[a];
-                if (F + warp_sum_u64(sl) >= T) lo = mid; else hi = mid;
-            }
-            // v = q of the free energy whose pattern is lo (it exists and has q > 0)
-            uint64_t vl = 0;
-#pragma unroll
-            for (int m = 0; m < MPL; ++m)
-                if (b[m] == lo && !((fbits >> m) & 1u)) vl = q[m] > vl ? q[m] : vl;
-            const uint64_t v = warp_max_u64(vl);
-            uint64_t gl = 0;
-#pragma unroll
-            for (int m = 0; m < MPL; ++m)
-                if (!((fbits >> m) & 1u) && q[m] > v) { gl += q[m]; kbits |= 1u << m; }
-            const uint64_t R = T - F - warp_sum_u64(gl);                 // > 0
-            const uint64_t need = (R + v - 1) / v;
-            uint64_t taken = 0;
+        if (__any_sync(0xffffffffu, bad) && lane == 0) raise_status(STATUS_BAD_ENERGY);
+        xmax = warp_max_u32(xmax);
+
+        uint32_t kbits = fbits;
+        if (xmax == 0u) {
+            const int jd = i < nk ? i : 0;                   // all-zero row
+            if (jd >= j0 && jd < j0 + MPL) kbits |= 1u << (jd - j0);
+        } else {
+            const int shift = 52 - float_exponent_p(xmax) - c;
+            uint32_t ql[MPL], qh[MPL];
+            uint32_t al = 0, ah = 0, fl = 0, fh = 0, bmax = 0;
 #pragma unroll
             for (int m = 0; m < MPL; ++m) {
-                const bool eq = !((fbits >> m) & 1u) && q[m] == v && static_cast<int>(lane) + 32 * m < nk;
-                const uint32_t ball = __ballot_sync(0xffffffffu, eq);
-                const uint64_t rank = taken + __popc(ball & lanemask_lt());
-                if (eq && rank < need) kbits |= 1u << m;
-                taken += __popc(ball);
+                const uint64_t q = quantize_bits(b[m], shift);
+                ql[m] = static_cast<uint32_t>(q) & lomask;
+                qh[m] = static_cast<uint32_t>(q >> cs);
+                al += ql[m];
+                ah += qh[m];
+                if ((fbits >> m) & 1u) {
+                    fl += ql[m];
+                    fh += qh[m];
+                    b[m] = 0u;                               // forced blocks are not free
+                }
+                bmax = b[m] > bmax ? b[m] : bmax;
+            }
+            const uint64_t Q = join(warp_sum_u32(ah), warp_sum_u32(al));
+            const uint64_t F = join(warp_sum_u32(fh), warp_sum_u32(fl));
+            bmax = warp_max_u32(bmax);
+            uint64_t T = __double2ull_rz(ceil(__dmul_rn(p.tau[bi], __ull2double_rn(Q))));
+            if (T < 1) T = 1;
+            if (F < T) {
+                // G(u) over every free element of the row (u >= 1: forced and padding have b = 0)
+                auto G_all = [&](uint32_t u) -> uint64_t {
+                    uint32_t sl = 0, sh = 0;
+#pragma unroll
+                    for (int m = 0; m < MPL; ++m) {
+                        const bool in = b[m] >= u;
+                        sl += in ? ql[m] : 0u;
+                        sh += in ? qh[m] : 0u;
+                    }
+                    return F + join(warp_sum_u32(sh), warp_sum_u32(sl));
+                };
+                // 1. exponent level: G(0) = Q >= T, G((lvl(bmax)+1) << 23) = F < T
+                uint32_t lo = 0, hi = (bmax >> 23) + 1;
+                uint64_t A = F;                              // G(hi << 23)
+                while (hi - lo > 1) {
+                    const uint32_t mid = (lo + hi) >> 1;
+                    const uint64_t g = G_all(mid << 23);
+                    if (g >= T) lo = mid;
+                    else { hi = mid; A = g; }
+                }
+                const uint32_t lvl = lo;
+                // 2. low bits inside the level
+                uint32_t ul = lvl << 23, uh = (lvl + 1) << 23;
+                uint32_t cl = 0;
+#pragma unroll
+                for (int m = 0; m < MPL; ++m) cl += (b[m] != 0u && (b[m] >> 23) == lvl) ? 1u : 0u;
+                const uint32_t nc = warp_sum_u32(cl);
+                if (nc <= static_cast<uint32_t>(kSelCompact)) {
+                    uint32_t pos = warp_exclusive_scan(cl);
+#pragma unroll
+                    for (int m = 0; m < MPL; ++m) {
+                        if (b[m] != 0u && (b[m] >> 23) == lvl) {
+                            cand_b[wib][pos] = b[m];
+                            cand_l[wib][pos] = ql[m];
+                            cand_h[wib][pos] = qh[m];
+                            ++pos;
+                        }
+                    }
+                    __syncwarp();
+                    const bool v0 = lane < nc, v1 = lane + 32 < nc;
+                    const uint32_t b0 = v0 ? cand_b[wib][lane] : 0u, b1 = v1 ? cand_b[wib][lane + 32] : 0u;
+                    const uint32_t l0 = v0 ? cand_l[wib][lane] : 0u, l1 = v1 ? cand_l[wib][lane + 32] : 0u;
+                    const uint32_t h0 = v0 ? cand_h[wib][lane] : 0u, h1 = v1 ? cand_h[wib][lane + 32] : 0u;
+                    __syncwarp();
+                    // G(u) = A + (level elements with b >= u), for u inside the level
+                    while (uh - ul > 1) {
+                        const uint32_t mid = ul + ((uh - ul) >> 1);
+                        const uint32_t sl = (b0 >= mid ? l0 : 0u) + (b1 >= mid ? l1 : 0u);
+                        const uint32_t sh = (b0 >= mid ? h0 : 0u) + (b1 >= mid ? h1 : 0u);
+                        if (A + join(warp_sum_u32(sh), warp_sum_u32(sl)) >= T) ul = mid;
+                        else uh = mid;
+                    }
+                } else {
+                    while (uh - ul > 1) {
+                        const uint32_t mid = ul + ((uh - ul) >> 1);
+                        if (G_all(mid) >= T) ul = mid;
+                        else uh = mid;
+                    }
+                }
+                const uint64_t v = quantize_bits(ul, shift);    // > 0 (see above)
+                // free blocks above v are kept; ties at v are taken in index order
+                uint32_t gl = 0, gh = 0, ce = 0;
+                uint32_t eqbits = 0;
+#pragma unroll
+                for (int m = 0; m < MPL; ++m) {
+                    const uint64_t q = (static_cast<uint64_t>(qh[m]) << cs) | ql[m];
+                    const bool fr = !((fbits >> m) & 1u) && j0 + m < nk;
+                    if (fr && q > v) {
+                        kbits |= 1u << m;
+                        gl += ql[m];
+                        gh += qh[m];
+                    } else if (fr && q == v) {
+                        eqbits |= 1u << m;
+                        ++ce;
+                    }
+                }
+                const uint64_t R = T - F - join(warp_sum_u32(gh), warp_sum_u32(gl));   // > 0
+                uint64_t need = v ? static_cast<uint64_t>(ceil(__ddiv_rn(__ull2double_rn(R), __ull2double_rn(v))))
+                                  : 0ull;
+                if (v) {
+                    while (need * v < R) ++need;                   // exact ceil(R / v)
+                    while (need > 0 && (need - 1) * v >= R) --need;
+                }
+                uint64_t rank = warp_exclusive_scan(ce);
+#pragma unroll
+                for (int m = 0; m < MPL; ++m) {
+                    if ((eqbits >> m) & 1u) {
+                        if (rank < need) kbits |= 1u << m;
+                        ++rank;
+                    }
+                }
             }
         }
-    } else {
-        const int jd = i < nk ? i : 0;                                   // all-zero row
-        if ((jd & 31) == static_cast<int>(lane)) kbits |= 1u << (jd >> 5);
-    }
+        if (p.mask_out) {
+            uint8_t* M = p.mask_out + (static_cast<size_t>(bi) * p.rows + row) * nk;
+            if constexpr (MPL % 4 == 0) {
+                if (p.vec) {
 #pragma unroll
-    for (int m = 0; m < MPL; ++m) {
-        const int j = static_cast<int>(lane) + 32 * m;
-        if (j < nk) {
-            const uint8_t k = static_cast<uint8_t>((kbits >> m) & 1u);
-            mask_out[base + j] = k;
-            if (count_accum) count_accum[base + j] += k;
+                    for (int v = 0; v < MPL / 4; ++v) {
+                        if (j0 + 4 * v < nk) {
+                            const uint32_t x = (kbits >> (4 * v)) & 0xFu;
+                            reinterpret_cast<uint32_t*>(M + j0)[v] =
+                                (x & 1u) | ((x & 2u) << 7) | ((x & 4u) << 14) | ((x & 8u) << 21);
+                        }
+                    }
+                }
+            }
+            if (!(MPL % 4 == 0) || !p.vec) {
+#pragma unroll
+                for (int m = 0; m < MPL; ++m)
+                    if (j0 + m < nk) M[j0 + m] = static_cast<uint8_t>((kbits >> m) & 1u);
+            }
+        }
+#pragma unroll
+        for (int m = 0; m < MPL; ++m) cnt[m >> 2] += ((kbits >> m) & 1u) << (8 * (m & 3));
+    }
+    if (p.count_accum) {
+#pragma unroll
+        for (int m = 0; m < MPL; ++m) {
+            const uint32_t k = (cnt[m >> 2] >> (8 * (m & 3))) & 0xFFu;
+            if (k && j0 + m < nk) atomicAdd(p.count_accum + rbase + j0 + m, static_cast<int>(k));
         }
     }
+}
+
+// Energy-mean aggregation over calibration inputs: mean = sum / n, elementwise, with the
+// correctly rounded fp32 division.
+__global__ void __launch_bounds__(256)
+energy_mean_kernel(const float* __restrict__ sum, long long count, float n, float* __restrict__ mean) {
+    const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+    const long long t0 = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+    const bool vec = ((reinterpret_cast<uintptr_t>(sum) | reinterpret_cast<uintptr_t>(mean)) & 15u) == 0;
+    long long done = 0;
+    if (vec) {
+        const long long n4 = count / 4;
+        for (long long x = t0; x < n4; x += stride) {
+            const float4 s = reinterpret_cast<const float4*>(sum)[x];
+            reinterpret_cast<float4*>(mean)[x] =
+                make_float4(__fdiv_rn(s.x, n), __fdiv_rn(s.y, n), __fdiv_rn(s.z, n), __fdiv_rn(s.w, n));
+        }
+        done = n4 * 4;
+    }
+    for (long long x = done + t0; x < count; x += stride) mean[x] = __fdiv_rn(sum[x], n);
 }
 
 // Cross-input vote, one warp per row: keep iff count * rho_den > rho_num * n_inputs;

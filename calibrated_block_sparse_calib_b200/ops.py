@@ -41,6 +41,9 @@ _SIGS = {
     "calib_device_check": ([_P], ctypes.c_int),
     "calib_block_energy": ([_P, _P, _P, _I, _I, _I, _I, _F, _P, _I, _P, _I, _P], ctypes.c_int),
     "calib_select_mask": ([_P, _I, _I, _I, _D, _P, _P, _P, _P], ctypes.c_int),
+    "calib_select_mask_batched": ([_P, _I, _I, _I, _I, _P, _P, _P, _P, _P], ctypes.c_int),
+    "calib_energy_mean": ([_P, ctypes.c_int64, _I, _P, _P], ctypes.c_int),
+    "calib_validate_block_list_host": ([_I, _I, _I, _P, _P, ctypes.c_int64, _P, _I], ctypes.c_int),
     "calib_aggregate_masks": ([_P, _I, _I, _I, _I, _I, _I, _P, _P], ctypes.c_int),
     "calib_mask_to_csr": ([_P, _I, _I, _I, _P, _P, _P], ctypes.c_int),
     "calib_build_schedule": ([_P, _I, _I, _P, _P], ctypes.c_int),
@@ -162,6 +165,65 @@ def select_mask(energy: torch.Tensor, tau: float, force_keep: Optional[torch.Ten
     _check("calib_select_mask", lib().calib_select_mask(
         _ptr(energy), H, nq, nk, float(tau), _ptr(force_keep), _ptr(out), _ptr(count_accum), _stream()))
     return out
+
+
+def select_mask_batched(energy: torch.Tensor, taus: Sequence[float], force_keep: Optional[torch.Tensor] = None,
+                        out: Optional[torch.Tensor] = None, count_accum: Optional[torch.Tensor] = None,
+                        write_masks: bool = True) -> Optional[torch.Tensor]:
+    """Minimal tau-energy selection of a batch energy[b] (fp32 [nb, H, nq, nk]) at taus[b], in
+    one launch.  Returns the uint8 masks [nb, H, nq, nk] (None with write_masks=False, when
+    only count_accum [H, nq, nk] is wanted: it is incremented by the number of entries that
+    keep each block)."""
+    _need(energy, "energy", torch.float32)
+    nb, H, nq, nk = energy.shape
+    taus = [float(t) for t in taus]
+    if len(taus) != nb:
+        raise ValueError(f"need one tau per batch entry ({nb}), got {len(taus)}")
+    if force_keep is not None:
+        _need(force_keep, "force_keep", torch.uint8, (H, nq, nk))
+    if count_accum is not None:
+        _need(count_accum, "count_accum", torch.int32, (H, nq, nk))
+    if write_masks:
+        if out is None:
+            out = torch.empty(energy.shape, dtype=torch.uint8, device=energy.device)
+        _need(out, "out", torch.uint8, energy.shape)
+    else:
+        out = None
+        if count_accum is None:
+            raise ValueError("write_masks=False needs count_accum")
+    tau_arr = (ctypes.c_double * nb)(*taus)
+    _check("calib_select_mask_batched", lib().calib_select_mask_batched(
+        _ptr(energy), nb, H, nq, nk, ctypes.cast(tau_arr, ctypes.c_void_p), _ptr(force_keep), _ptr(out),
+        _ptr(count_accum), _stream()))
+    return out
+
+
+def energy_mean(energy_sum: torch.Tensor, n_inputs: int, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """fp32 energies averaged over n_inputs calibration inputs (energy_sum / n_inputs); `out`
+    may be energy_sum itself."""
+    _need(energy_sum, "energy_sum", torch.float32)
+    if out is None:
+        out = torch.empty_like(energy_sum)
+    _need(out, "out", torch.float32, energy_sum.shape)
+    _check("calib_energy_mean", lib().calib_energy_mean(
+        _ptr(energy_sum), energy_sum.numel(), int(n_inputs), _ptr(out), _stream()))
+    return out
+
+
+def validate_block_list_host(H: int, nq: int, nk: int, row_ptr, col_idx, work=None) -> bool:
+    """True when a skip list held in host memory (numpy arrays or CPU tensors) is well formed
+    for the attention calls (calib_validate_block_list_host); no device work."""
+    import numpy as np
+    rp = np.ascontiguousarray(np.asarray(row_ptr), dtype=np.int32)
+    ci = np.ascontiguousarray(np.asarray(col_idx), dtype=np.int16)
+    if rp.shape != (H * nq + 1,):
+        return False
+    wk = None if work is None else np.ascontiguousarray(np.asarray(work), dtype=np.int32)
+    s = lib().calib_validate_block_list_host(
+        int(H), int(nq), int(nk), rp.ctypes.data_as(ctypes.c_void_p),
+        ci.ctypes.data_as(ctypes.c_void_p) if ci.size else None, int(ci.size),
+        None if wk is None else wk.ctypes.data_as(ctypes.c_void_p), 0 if wk is None else int(wk.size))
+    return s == CALIB_OK
 
 
 def aggregate_masks(counts: torch.Tensor, n_inputs: int, rho: Sequence[int] = (1, 2),
@@ -299,6 +361,15 @@ class BlockList:
         return _BlockListC(self.H, self.nq, self.nk, self.block, self.row_ptr.data_ptr(),
                            self.col_idx.data_ptr(), 0 if self.work is None else self.work.data_ptr(),
                            0 if self.work is None else self.work.numel())
+
+    def validate(self) -> "BlockList":
+        """Copy the list back to the host and check its structure (rows within col_idx,
+        ascending in-range indices, work items in range); raises ValueError if malformed."""
+        H, nq, nk = self.H, self.nq, self.nk
+        wk = None if self.work is None else self.work.cpu().numpy()
+        if not validate_block_list_host(H, nq, nk, self.row_ptr.cpu().numpy(), self.col_idx.cpu().numpy(), wk):
+            raise ValueError("malformed skip list")
+        return self
 
     @staticmethod
     def from_mask(mask: torch.Tensor, block: int, schedule: bool = True) -> "BlockList":

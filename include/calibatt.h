@@ -72,9 +72,11 @@ const char* calib_status_string(calib_status s);
 
 /* Synchronises `stream`, then reads and clears the status word of the current device.
  * Returns CALIB_ERR_TIMEOUT if any kernel since the last check gave up on a bounded
- * wait, CALIB_ERR_INVALID if a selection kernel met a negative or non-finite energy
- * (treated as 0), CALIB_ERR_CUDA on a CUDA error (or a kernel that found its shared
- * memory misaligned and did nothing), else CALIB_OK. */
+ * wait; CALIB_ERR_INVALID if a selection kernel met a negative or non-finite energy
+ * (treated as 0) or an attention kernel met a work item outside the call (head >= H or
+ * query block >= nq) or a skip-list row with a negative start, decreasing pointers or
+ * more than nk blocks (that item is skipped, its output rows are not written);
+ * CALIB_ERR_CUDA on a CUDA error; else CALIB_OK. */
 calib_status calib_device_check(void* stream);
 
 /* Row log-sum-exp and block energies, fused ([zh] §2.2A, [de] §2A.1, [fr] §2.B.1: split
@@ -98,7 +100,8 @@ calib_status calib_block_energy(const void* q, const void* k, const float* lse,
                                 float* energy, int accumulate, void* stream);
 
 /* Minimal tau-energy selection ([fr] §2.B.1: per query block, the fewest key blocks whose
- * cumulative energy reaches the threshold; [zh] §2.2A, [de] §2A.2), one warp per row:
+ * cumulative energy reaches the threshold; [zh] §2.2A, [de] §2A.2), one warp per row.
+ * Equivalent to calib_select_mask_batched with one batch entry:
  *   energy     : fp32 [H, nq, nk], finite and >= 0.
  *   tau        : in (0, 1]; the per-timestep threshold eps(t).
  *   force_keep : NULL or uint8 [H, nq, nk]; forced blocks are kept first and count
@@ -114,6 +117,35 @@ calib_status calib_block_energy(const void* q, const void* k, const float* lse,
 calib_status calib_select_mask(const float* energy, int H, int nq, int nk, double tau,
                                const uint8_t* force_keep, uint8_t* mask_out,
                                int32_t* count_accum, void* stream);
+
+/* Minimal tau-energy selection over a batch of energy matrices in one launch: the rows of
+ * every (calibration input, timestep) pair of a calibration slice or sweep ([fr] §2.B.1:
+ * one selection per query block at the timestep's threshold eps(t)).
+ *   energy      : fp32 [nb, H, nq, nk], finite and >= 0; entry b is selected at tau[b].
+ *   nb          : 1 .. 256 entries.
+ *   tau         : HOST double [nb], each in (0, 1].
+ *   force_keep  : NULL or uint8 [H, nq, nk], shared by every entry.
+ *   mask_out    : NULL or uint8 [nb, H, nq, nk], the mask of every entry.
+ *   count_accum : NULL or int32 [H, nq, nk]; each (h, i, j) is incremented by the number of
+ *                 entries that keep it (the vote counts of calib_aggregate_masks when the
+ *                 entries are one slice's calibration inputs).  Increments are atomic, so
+ *                 the result does not depend on the order in which entries are processed.
+ * At least one of mask_out and count_accum must be given.  The rule and its integer
+ * arithmetic are those of calib_select_mask, row by row and entry by entry.  Energy and
+ * count_accum pointers must be 4-byte aligned.  nk <= 1024. */
+calib_status calib_select_mask_batched(const float* energy, int nb, int H, int nq, int nk,
+                                       const double* tau, const uint8_t* force_keep,
+                                       uint8_t* mask_out, int32_t* count_accum, void* stream);
+
+/* Energy-mean aggregation over calibration inputs: the block energies averaged over the
+ * inputs, then selected once (the alternative to the pages' vote over per-input masks,
+ * calib_aggregate_masks; with one input both give that input's mask):
+ *   mean_out[x] = energy_sum[x] / n_inputs,  x < count,
+ * in fp32 with a correctly rounded division.  energy_sum is the fp32 sum of the inputs'
+ * energies, as calib_block_energy(accumulate = 1) leaves it; mean_out may be energy_sum
+ * (in place).  Pointers 4-byte aligned; 1 <= n_inputs <= 2^24. */
+calib_status calib_energy_mean(const float* energy_sum, int64_t count, int n_inputs,
+                               float* mean_out, void* stream);
 
 /* Cross-input vote ([zh] §2.2A, [de] §2A.3, [fr] §2.B.2): keep (h, i, j) iff
  * counts[h,i,j] * rho_den > rho_num * n_inputs (frequency strictly above rho =
@@ -204,7 +236,8 @@ calib_status calib_anchor_rows(int F, int Hl, int Wl, int n_text, int stride,
  * rounded to bf16 for the PV product and O is divided by the sum of those rounded
  * weights.
  * A row with no kept block writes O = 0 and LSE = -inf.  With an all-kept list this is
- * dense attention. */
+ * dense attention.  The list is trusted: calib_validate_block_list_host checks one that
+ * comes from outside the library's own builders. */
 calib_status sparse_attn_fwd(const void* q, const void* k, const void* v, void* o,
                              float* lse_opt, int H, int N, int D, float scale,
                              const calib_block_list* list, uint32_t flags, void* stream);
@@ -259,6 +292,23 @@ calib_status sparse_attn_fwd_repeat(const void* q, const void* k, const void* v,
                                     int n_text, int stride, const uint8_t* head_repeat,
                                     float scale, const calib_block_list* list,
                                     uint32_t flags, void* stream);
+
+/* Checks a skip list held in HOST memory (copied back from the device by the caller) before
+ * it is given to the attention calls, which trust the list's structure: row_ptr[0] == 0;
+ * for every row r < H*nq, row_ptr[r] <= row_ptr[r+1] <= col_capacity and the row keeps at
+ * most nk blocks; each row's col_idx strictly ascending in [0, nk); and, when `work` is
+ * given, every entry h << 16 | i with 0 <= h < H and 0 <= i < nq.  ([fr] §2.C: the lists
+ * are precomputed and held in memory before inference; a list that comes from elsewhere is
+ * checked here.)
+ *   row_ptr     : HOST int32 [H*nq + 1].
+ *   col_idx     : HOST int16, col_capacity entries (may be NULL when the list is empty).
+ *   work        : HOST int32 [n_work] or NULL.
+ * Pure host code, no device work: returns CALIB_OK or CALIB_ERR_INVALID.  The attention
+ * kernels themselves skip (and report through calib_device_check) items whose head, query
+ * block or row pointers are out of range, but they cannot see col_idx's capacity. */
+calib_status calib_validate_block_list_host(int H, int nq, int nk, const int32_t* row_ptr,
+                                            const int16_t* col_idx, int64_t col_capacity,
+                                            const int32_t* work, int n_work);
 
 /* Failure-detection self-test: launches one kernel that waits, with the library's bounded
  * wait, on an mbarrier that nothing ever completes, giving up after timeout_us

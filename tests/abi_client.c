@@ -75,6 +75,32 @@ int main(void) {
                                        rep, 0.1f, &bl_bad, 0, 1, NULL, NULL, NULL) == CALIB_ERR_INVALID,
            "host repeat list shape");
 
+    /* batched selection: no output, too many entries, a tau outside (0, 1] */
+    {
+        double taus[2] = {0.9, 1.5};
+        expect(calib_select_mask_batched((const float*)fake, 1, 1, 1, 1, taus, NULL, NULL, NULL, NULL) ==
+                   CALIB_ERR_INVALID, "batched select without outputs");
+        expect(calib_select_mask_batched((const float*)fake, 257, 1, 1, 1, taus, NULL, (uint8_t*)fake, NULL, NULL) ==
+                   CALIB_ERR_INVALID, "batched select 257 entries");
+        expect(calib_select_mask_batched((const float*)fake, 2, 1, 1, 1, taus, NULL, (uint8_t*)fake, NULL, NULL) ==
+                   CALIB_ERR_INVALID, "batched select tau 1.5");
+    }
+    /* energy mean: zero inputs */
+    expect(calib_energy_mean((const float*)fake, 4, 0, (float*)fake, NULL) == CALIB_ERR_INVALID, "mean 0 inputs");
+
+    /* host-side skip-list check: a valid 2 x 2 list, then an index past nk and a bad work item */
+    {
+        int32_t rp2[3] = {0, 2, 3};
+        int16_t ci2[3] = {0, 1, 1};
+        int32_t wk[2] = {1, 0};
+        int32_t wk_bad[2] = {1, 2};
+        int16_t ci_bad[3] = {0, 2, 1};
+        expect(calib_validate_block_list_host(1, 2, 2, rp2, ci2, 3, wk, 2) == CALIB_OK, "valid list");
+        expect(calib_validate_block_list_host(1, 2, 2, rp2, ci_bad, 3, wk, 2) == CALIB_ERR_INVALID, "index >= nk");
+        expect(calib_validate_block_list_host(1, 2, 2, rp2, ci2, 3, wk_bad, 2) == CALIB_ERR_INVALID, "work i >= nq");
+        expect(calib_validate_block_list_host(1, 2, 2, rp2, ci2, 2, wk, 2) == CALIB_ERR_INVALID, "beyond capacity");
+    }
+
     if (failures == 0) printf("ok\n");
     return failures == 0 ? 0 : 1;
 }

@@ -100,6 +100,65 @@ def test_bad_headers_are_refused():
         with pytest.raises(ValueError):
             MaskDictionary.from_bytes(bytes(b), device="cpu")
     b = bytearray(buf)
-    struct.pack_into("<i", b, 40 + 8, -5)                # a negative run count
+    struct.pack_into("<i", b, 64 + 8, -5)                # a negative run count
     with pytest.raises(ValueError):
         MaskDictionary.from_bytes(bytes(b), device="cpu")
+    for field, value in ((8, 3), (9, 0), (10, 7), (11, -1)):   # rho 3/2, rho_den 0, mode 7, n_inputs -1
+        b = bytearray(buf)
+        struct.pack_into("<i", b, 8 + 4 * field, value)
+        if field == 8:
+            struct.pack_into("<i", b, 8 + 4 * 9, 2)
+        with pytest.raises(ValueError):
+            MaskDictionary.from_bytes(bytes(b), device="cpu")
+    b = bytearray(buf)
+    struct.pack_into("<d", b, 64 + 12, 1.5)              # a slice tau above 1
+    with pytest.raises(ValueError):
+        MaskDictionary.from_bytes(bytes(b), device="cpu")
+
+
+def test_calibration_record_round_trips():
+    """The file says how it was calibrated: the vote threshold rho, the aggregation mode,
+    the number of inputs, the repetition threshold gamma and every slice's tau."""
+    d, ref = _dict(3)
+    d.rho, d.mode, d.n_inputs, d.gamma = (2, 3), "energy_mean", 4, 0.9
+    for n, key in enumerate(sorted(d.slices)):
+        d.slices[key].tau = [0.99, 0.95, 0.9][n % 3]
+    e = MaskDictionary.from_bytes(d.to_bytes(), device="cpu")
+    assert (e.rho, e.mode, e.n_inputs, e.gamma) == ((2, 3), "energy_mean", 4, 0.9)
+    for n, key in enumerate(sorted(ref)):
+        assert e.tau(*key) == [0.99, 0.95, 0.9][n % 3]
+    d.gamma = None
+    d.mode = "given"
+    e = MaskDictionary.from_bytes(d.to_bytes(), device="cpu")
+    assert e.gamma is None and e.mode == "given"
+
+
+def test_first_format_is_refused_with_a_reason():
+    d, _ = _dict(4)
+    buf = b"CBSDICT1" + d.to_bytes()[8:]
+    with pytest.raises(ValueError, match="CBSDICT1.*no calibration parameters"):
+        MaskDictionary.from_bytes(buf, device="cpu")
+
+
+def test_truncated_files_name_what_is_missing():
+    d, _ = _dict(5)
+    buf = d.to_bytes()
+    for cut in (12, 60, 64 + 10, 64 + 20 + 3, len(buf) // 2, len(buf) - 2):
+        with pytest.raises(ValueError, match="truncated|trailing|offsets|run"):
+            MaskDictionary.from_bytes(buf[:cut], device="cpu")
+    for cut in (12, 60, 64 + 10, 64 + 20 + 3):
+        with pytest.raises(ValueError, match="truncated"):
+            MaskDictionary.from_bytes(buf[:cut], device="cpu")
+
+
+def test_skip_lists_beyond_int32_offsets_are_refused():
+    """70000 rows, each one run of 32767 blocks: under 1 MB on disk, but the expanded skip
+    list would hold 2.3e9 entries, past the int32 row offsets the device kernels use."""
+    H, nq, nk = 1, 70000, 32767
+    iv_ptr = np.arange(nq + 1, dtype="<i4")
+    runs = np.zeros(nq, "<i2").tobytes() + np.full(nq, nk, "<i2").tobytes()
+    buf = (MAGIC + struct.pack("<12i", 1, 1, H, nq, nk, 128, 1, 1, 1, 2, 0, 1) + struct.pack("<d", float("nan")) +
+           struct.pack("<3id", 0, 0, nq, 0.9) + b"\1\0\0\0" + iv_ptr.tobytes() + runs)
+    assert len(buf) < 1 << 20
+    with pytest.raises(ValueError, match="2\\^31"):
+        MaskDictionary.from_bytes(buf, device="cpu")

@@ -140,6 +140,69 @@ def test_select_forced_and_count_accumulation():
     np.testing.assert_array_equal(counts.cpu().numpy(), acc)
 
 
+def _hard_rows(rng, H, nq, nk):
+    """Rows that stress the selection kernel's two search paths: the answer's exponent level
+    holding 1, ~20, ~50 (two per lane) or all of the row's blocks (equal energies), blocks of
+    -0.0, and values straddling a power of two."""
+    e = _energy_rows(rng, H, nq, nk).astype(np.float64)
+    for h in range(H):
+        for i in range(nq):
+            kind = (h * nq + i) % 5
+            if kind == 0:
+                e[h, i] = 0.25                                     # all equal
+            elif kind == 1:
+                x = np.full(nk, 2.0 ** -20)
+                x[rng.choice(nk, size=min(nk, 50), replace=False)] = 1.0 + rng.random(min(nk, 50)) * 0.5
+                e[h, i] = x
+            elif kind == 2:
+                x = rng.random(nk) * 0.01
+                x[rng.choice(nk, size=min(nk, 20), replace=False)] = 1.0 + rng.random(min(nk, 20))
+                e[h, i] = x
+            elif kind == 3:
+                e[h, i] = np.where(rng.random(nk) < 0.5, 1.0, 1.0 - 2.0 ** -24)      # either side of 2^0
+    e = e.astype(np.float32)
+    e[0, 0, :: 3] = np.float32(-0.0)
+    return e
+
+
+@pytest.mark.parametrize("nk", [1, 2, 33, 64, 100, 256, 591, 1024])
+def test_select_batched_bit_exact(nk):
+    """One launch over nb entries, each at its own tau, with shared forced blocks, per-entry
+    masks and vote counts: every entry's mask equals the oracle's selection of that entry,
+    and the counts equal the sum of the masks."""
+    rng = np.random.default_rng(1000 + nk)
+    taus = [1e-7, 0.5, 0.9, 0.95, 0.99, 1.0]
+    H, nq = 2, 5
+    e = np.stack([_hard_rows(rng, H, nq, nk) for _ in taus])
+    force = (rng.random((H, nq, nk)) < 0.03).astype(np.uint8)
+    counts = torch.full((H, nq, nk), 7, dtype=torch.int32, device="cuda")    # counts add to what is there
+    got = ops.select_mask_batched(torch.from_numpy(e).cuda(), taus, force_keep=torch.from_numpy(force).cuda(),
+                                  count_accum=counts).cpu().numpy()
+    acc = np.full((H, nq, nk), 7, np.int64)
+    for b, tau in enumerate(taus):
+        ref = oracle.select_mask(e[b], tau, force_keep=force)
+        np.testing.assert_array_equal(got[b], ref, err_msg=f"entry {b} tau {tau}")
+        acc += ref
+    np.testing.assert_array_equal(counts.cpu().numpy(), acc)
+    ops.device_check()
+
+
+def test_select_batched_many_entries_split_over_warps():
+    """Enough rows x entries that each row's entries are split into chunks handled by
+    different warps (vote counts then combine atomically); counts only, no masks."""
+    rng = np.random.default_rng(77)
+    nb, H, nq, nk = 20, 4, 250, 64
+    e = np.stack([_energy_rows(rng, H, nq, nk) for _ in range(nb)])
+    taus = [0.8 + 0.01 * b for b in range(nb)]
+    counts = torch.zeros((H, nq, nk), dtype=torch.int32, device="cuda")
+    assert ops.select_mask_batched(torch.from_numpy(e).cuda(), taus, count_accum=counts, write_masks=False) is None
+    acc = sum(oracle.select_mask(e[b], taus[b]).astype(np.int64) for b in range(nb))
+    np.testing.assert_array_equal(counts.cpu().numpy(), acc)
+    masks = ops.select_mask_batched(torch.from_numpy(e).cuda(), taus).cpu().numpy()
+    for b in (0, 7, 19):
+        np.testing.assert_array_equal(masks[b], oracle.select_mask(e[b], taus[b]))
+
+
 @pytest.mark.parametrize("n_inputs,rho", [(1, (1, 2)), (3, (1, 2)), (4, (1, 2)), (5, (1, 3)), (4, (0, 1))])
 def test_aggregate_bit_exact(n_inputs, rho):
     rng = np.random.default_rng(n_inputs * 7 + rho[0])
@@ -268,9 +331,41 @@ def test_energy_cached_lse_and_accumulate(tiny_inputs):
     lse_t = torch.from_numpy(lse.astype(np.float32)).cuda()
     got = ops.block_energy(q.cuda(), k.cuda(), B, lse=lse_t)
     check_energy(got, ref, wl.shape.N, B)
-    acc = ops.block_energy(q.cuda(), k.cuda(), B, accumulate=True)
-    acc = ops.block_energy(q.cuda(), k.cuda(), B, out=acc, accumulate=True)
-    check_energy(acc, 2 * ref, wl.shape.N, B)
+
+
+def test_energy_accumulate_and_mean_over_three_distinct_inputs(tiny_inputs):
+    """The energy-mean aggregation: the accumulate flag sums three DIFFERENT inputs'
+    energies, calib_energy_mean divides by the input count, and both match the oracle's
+    float64 sum and mean (energy_mean) within the energy tolerance.  Selection on the GPU's
+    mean energies is bit-exact against the oracle's selection on the same energies."""
+    wl, qkv = tiny_inputs
+    B, D, N = wl.shape.block, wl.shape.D, wl.shape.N
+    scale = 1.0 / math.sqrt(D)
+    refs = [oracle.block_energy(to64(q), to64(k), scale, B) for q, k, _ in qkv]
+    assert len(refs) == 3 and not np.allclose(refs[0], refs[1])
+    acc = None
+    for d, (q, k, _) in enumerate(qkv):
+        acc = ops.block_energy(q.cuda(), k.cuda(), B, out=acc, accumulate=d > 0)
+        check_energy(acc, sum(refs[:d + 1]), N, B)               # each partial sum
+    esum = acc.clone()
+    mean = ops.energy_mean(acc, len(qkv))
+    check_energy(mean, oracle.energy_mean(refs).astype(np.float64), N, B)
+    # the mean is the correctly rounded fp32 quotient of the fp32 sum
+    np.testing.assert_array_equal(mean.cpu().numpy(), esum.cpu().numpy() / np.float32(3))
+    inplace = ops.energy_mean(esum, len(qkv), out=esum)
+    assert inplace.data_ptr() == esum.data_ptr()
+    np.testing.assert_array_equal(inplace.cpu().numpy(), mean.cpu().numpy())
+    for tau in (0.5, 0.9, 0.95, 0.99):
+        got = ops.select_mask(mean, tau).cpu().numpy()
+        np.testing.assert_array_equal(got, oracle.select_mask(mean.cpu().numpy(), tau))
+
+
+@pytest.mark.parametrize("count", [1, 3, 4, 1001, 4096 * 33 + 2])
+def test_energy_mean_sizes(count):
+    rng = np.random.default_rng(count)
+    x = (rng.random(count) * 7).astype(np.float32)
+    got = ops.energy_mean(torch.from_numpy(x).cuda(), 7).cpu().numpy()
+    np.testing.assert_array_equal(got, x / np.float32(7))
 
 
 @pytest.mark.parametrize("geom", [(2, 64, 4, 8, 16, 64), (2, 128, 6, 10, 23, 128)])
@@ -450,7 +545,13 @@ def test_calibration_pipeline_tiny(tiny_inputs):
     np.testing.assert_array_equal(counts.cpu().numpy(), cnt_ref)
     agg = ops.aggregate_masks(counts, len(qkv), rho).cpu().numpy()
     np.testing.assert_array_equal(agg, oracle.aggregate_masks(cnt_ref, len(qkv), *rho))
-    # energy-mean mode: the sum of fp32 energies is what selection sees
+    # the same vote in one batched launch over the three inputs' energies
+    counts_b = torch.zeros_like(counts)
+    stack = torch.from_numpy(np.stack(energies_gpu)).cuda()
+    masks_b = ops.select_mask_batched(stack, [tau] * len(qkv), count_accum=counts_b).cpu().numpy()
+    np.testing.assert_array_equal(counts_b.cpu().numpy(), cnt_ref)
+    for d, e in enumerate(energies_gpu):
+        np.testing.assert_array_equal(masks_b[d], oracle.select_mask(e, tau))
     bl = _blist(agg, B)
     q, k, v = qkv[0]
     O_ref, _ = oracle.sparse_attention(to64(q), to64(k), to64(v), scale, B, agg)
@@ -644,6 +745,33 @@ def test_repeat_similarity_wan13b_shape_sampled():
     got = ops.repeat_similarity(q, k, torch.from_numpy(mem).cuda(), s.F, s.Hl, s.Wl, 4)
     ref = oracle.repeat_similarity(to64(q), to64(k), 1.0 / math.sqrt(s.D), mem, s.F, s.Hl, s.Wl, 4)
     np.testing.assert_allclose(to64(got), ref, atol=COS_ABS, rtol=0)
+
+
+def test_calibrate_slice_energy_mean_bit_exact_from_gpu_energies():
+    """The calibration driver in energy-mean mode on 3 distinct inputs: its slice mask equals
+    the oracle's selection on the GPU's mean energies, and those energies match the oracle's
+    float64 mean within the energy tolerance."""
+    from calibrated_block_sparse_calib_b200.calibrate import calibrate_slice
+    wl = _shape(2, 64, 4, 8, 16, 64)
+    s = wl.shape
+    B, tau = s.block, 0.9
+    inputs = [tuple(t.cuda() for t in synth.make_qkv(wl, seed=300 + d)[:2]) for d in range(3)]
+    force = np.zeros((2, s.nblk, s.nblk), np.uint8)
+    force[:, :, 0] = 1                                          # a forced key column
+    mask, repeat, _ = calibrate_slice(inputs, s.F, s.Hl, s.Wl, 0, B, tau, mode="energy_mean",
+                                      force_keep=torch.from_numpy(force).cuda())
+    assert repeat == [False, False]
+    esum = None
+    for d, (q, k) in enumerate(inputs):
+        esum = ops.block_energy(q, k, B, out=esum, accumulate=d > 0)
+    mean = ops.energy_mean(esum, 3).cpu().numpy()
+    ref_e = oracle.energy_mean([oracle.block_energy(to64(q), to64(k), 1.0 / math.sqrt(s.D), B) for q, k in inputs])
+    check_energy(torch.from_numpy(mean), ref_e.astype(np.float64), s.N, B)
+    np.testing.assert_array_equal(mask.cpu().numpy(), oracle.select_mask(mean, tau, force_keep=force))
+    # the vote mode's slice differs in general; both are valid calibrations of the slice
+    vote, _, _ = calibrate_slice(inputs, s.F, s.Hl, s.Wl, 0, B, tau, mode="vote")
+    cnt = sum(oracle.select_mask(ops.block_energy(q, k, B).cpu().numpy(), tau).astype(np.int64) for q, k in inputs)
+    np.testing.assert_array_equal(vote.cpu().numpy(), oracle.aggregate_masks(cnt, 3, 1, 2))
 
 
 def test_calibrate_slice_with_repeat_head_bit_exact_from_gpu_energies():
