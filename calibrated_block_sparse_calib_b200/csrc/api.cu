@@ -100,31 +100,29 @@ calib_status launch_status() {
 }
 
 // ---- attention ---------------------------------------------------------------------
+// A validated attention call: parameters and tensor maps (K, V, and Q as whole blocks and
+// as single rows for gathered anchor rows), launchable in slices of the work list.
+struct AttnCall {
+    calib::AttnParams p;
+    CUtensorMap tk, tv, tq, tq1;
+    int D, B, grid;
+};
+
 template <int D, int BLK, bool WITH_LSE>
-calib_status launch_attn(const CUtensorMap& tk, const CUtensorMap& tv,
-                         const calib::AttnParams& p, int grid, cudaStream_t st) {
-    constexpr int KST = 3, VST = 3;   // K / V ring depths
+calib_status launch_attn(const AttnCall& c, const calib::AttnParams& p, int grid, cudaStream_t st) {
+    constexpr int KST = 3, VST = 2;   // K / V ring depths (with the Q tile, 200 KB at D = B = 128)
     using L = calib::AttnSmem<D, BLK, KST, VST>;
     static_assert(L::BYTES <= 232448, "shared memory budget");
     auto* fn = calib::attn_fwd_kernel<D, BLK, KST, VST, WITH_LSE>;
     if (calib_status s = ensure_smem(reinterpret_cast<const void*>(fn), L::BYTES)) return s;
-    fn<<<grid, calib::kAttnThreads, L::BYTES, st>>>(tk, tv, p);
+    fn<<<grid, calib::kAttnThreads, L::BYTES, st>>>(c.tk, c.tv, c.tq, c.tq1, p);
     return launch_status();
 }
 
 template <int D, int BLK>
-calib_status launch_attn_lse(const CUtensorMap& tk, const CUtensorMap& tv,
-                             const calib::AttnParams& p, int grid, cudaStream_t st) {
-    return p.lse ? launch_attn<D, BLK, true>(tk, tv, p, grid, st) : launch_attn<D, BLK, false>(tk, tv, p, grid, st);
+calib_status launch_attn_lse(const AttnCall& c, const calib::AttnParams& p, int grid, cudaStream_t st) {
+    return p.lse ? launch_attn<D, BLK, true>(c, p, grid, st) : launch_attn<D, BLK, false>(c, p, grid, st);
 }
-
-// A validated attention call: parameters and tensor maps, launchable in slices of the
-// work list.
-struct AttnCall {
-    calib::AttnParams p;
-    CUtensorMap tk, tv;
-    int D, B, grid;
-};
 
 calib_status attn_prepare(const void* q, const void* k, const void* v, void* o, float* lse, int H, int N,
                           int D, float scale, const calib_block_list* list, const uint32_t* repeat_bits,
@@ -163,7 +161,9 @@ calib_status attn_prepare(const void* q, const void* k, const void* v, void* o, 
     c->D = D;
     c->B = B;
     c->grid = list->work ? list->n_work : H * nb;
-    if (!make_tmap(&c->tk, k, D, N, H, B) || !make_tmap(&c->tv, v, D, N, H, B)) return CALIB_ERR_CUDA;
+    if (!make_tmap(&c->tk, k, D, N, H, B) || !make_tmap(&c->tv, v, D, N, H, B) ||
+        !make_tmap(&c->tq, q, D, N, H, B) || !make_tmap(&c->tq1, q, D, N, H, 1))
+        return CALIB_ERR_CUDA;
     return CALIB_OK;
 }
 
@@ -174,10 +174,9 @@ calib_status attn_launch(const AttnCall& c, int first, int count, cudaStream_t s
     calib::AttnParams p = c.p;
     if (p.work) p.work += first;
     else if (first != 0 || count != c.grid) return CALIB_ERR_INVALID;
-    if (c.D == 128) return c.B == 128 ? launch_attn_lse<128, 128>(c.tk, c.tv, p, count, st)
-                                      : launch_attn_lse<128, 64>(c.tk, c.tv, p, count, st);
-    return c.B == 128 ? launch_attn_lse<64, 128>(c.tk, c.tv, p, count, st)
-                      : launch_attn_lse<64, 64>(c.tk, c.tv, p, count, st);
+    if (c.D == 128) return c.B == 128 ? launch_attn_lse<128, 128>(c, p, count, st)
+                                      : launch_attn_lse<128, 64>(c, p, count, st);
+    return c.B == 128 ? launch_attn_lse<64, 128>(c, p, count, st) : launch_attn_lse<64, 64>(c, p, count, st);
 }
 
 calib_status attn_common(const void* q, const void* k, const void* v, void* o, float* lse, int H, int N,
