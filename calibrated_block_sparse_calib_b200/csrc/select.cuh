@@ -9,7 +9,8 @@ namespace calib {
 constexpr int kSelMaxPerLane = 32;   // nk <= 32 * 32 = 1024 in selection
 constexpr int kSelMaxBatch = 256;    // energy matrices per selection call
 constexpr int kSelWarps = 4;         // warps per CTA of the selection kernel
-constexpr int kSelCompact = 64;      // largest candidate set moved to shared memory
+constexpr int kSelCompact = 64;      // largest candidate set decided in shared memory
+constexpr int kSelBins = 128;        // histogram bins: half exponent levels below the row maximum
 
 // Parameters of one batched selection call.  Batch entry b is the energy matrix
 // energy[b] of shape [rows, nk] (rows = H * nq); force_keep and count_accum are shared by
@@ -71,6 +72,47 @@ __device__ __forceinline__ uint64_t quantize_bits(uint32_t x, int shift) {
     return qt + ((rem > half || (rem == half && (qt & 1u))) ? 1u : 0u);
 }
 
+// A copy of x that the compiler cannot see through: a value recomputed from it is not
+// merged with (or hoisted to) an earlier computation, so no per-block results stay live
+// across a loop just to be reused.
+__device__ __forceinline__ int opaque(int x) {
+    int y;
+    asm volatile("mov.b32 %0, %1;" : "=r"(y) : "r"(x));
+    return y;
+}
+
+// 64-bit sum over the lanes of a warp (butterfly of 32-bit shuffles).
+__device__ __forceinline__ uint64_t warp_sum_u64(uint64_t v) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+    return v;
+}
+// Exclusive prefix sum of 64-bit values over the lanes of a warp.
+__device__ __forceinline__ uint64_t warp_exclusive_scan_u64(uint64_t v) {
+    const uint32_t lane = lane_id();
+    uint64_t x = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const uint64_t y = __shfl_up_sync(0xffffffffu, x, off);
+        if (lane >= static_cast<uint32_t>(off)) x += y;
+    }
+    return x - v;
+}
+
+// quantize_bits on the FP64 pipe: for a normal binary32 x (exponent field E >= 1) the
+// binary64 with exponent E + 896 + shift and x's significand is exactly e * 2^shift (no
+// overflow or underflow for shift in [-86, 200]); adding 2^52 rounds it to an integer, half
+// to even (e * 2^shift < 2^52 here), which is then the low 52 bits of the sum.  Subnormal x
+// take the integer path.  Same value as quantize_bits, in a handful of instructions.
+__device__ __forceinline__ uint64_t quantize_fast(uint32_t x, int shift) {
+    const uint32_t E = x >> 23;
+    if (E == 0u) return quantize_bits(x, shift);
+    const uint32_t hi = ((E + 896u + static_cast<uint32_t>(shift)) << 20) | ((x & 0x7FFFFFu) >> 3);
+    const double d = __hiloint2double(static_cast<int>(hi), static_cast<int>(x << 29));
+    const double r = __dadd_rn(d, 4503599627370496.0);           // + 2^52
+    return static_cast<uint64_t>(__double_as_longlong(r)) & 0xFFFFFFFFFFFFFull;
+}
+
 // Minimal tau-energy selection, one warp per (row, chunk of batch entries); lane l holds
 // key blocks [l*MPL, (l+1)*MPL) of the row (nk <= 32*MPL).  See calib_select_mask in
 // calibatt.h for the rule.  With q_j the row's integer energies (shift chosen so that the
@@ -78,26 +120,37 @@ __device__ __forceinline__ uint64_t quantize_bits(uint32_t x, int shift) {
 // blocks, every free block with q_j > v, and the first c free blocks (ascending j) with
 // q_j == v, where v is the largest value with F + sum_{free, q_j >= v} q_j >= T.
 //
-// Finding v.  For e >= 0 the binary32 bit pattern b is monotone in e, and q is monotone in
-// e, so with G(u) = F + sum_{free, b_j >= u} q_j the largest pattern u* with G(u*) >= T is
-// the pattern of a free energy whose q is exactly v (G changes only where an element with
-// q > 0 drops out).  u* is found in two bisections:
-//   1. over the exponent field: the largest level e with G(e << 23) >= T (at most 8 steps
-//      over all of the row's elements);
-//   2. over the 23 low bits inside that level, where only the elements of that level can
-//      change G; when they are few (<= 64, the usual case: a factor-of-two band of
-//      energies) they are first moved to shared memory, two per lane, so each step
-//      touches two values instead of MPL.
-// Every sum is exact: q_j < 2^(52-c) with c = ceil(log2 nk) is split at bit 32-c into a
-// low part (row total < 2^32) and a high part (row total < 2^30), each reduced over the
-// warp with one 32-bit redux.
+// For e >= 0 the binary32 bit pattern b is monotone in e, and q is monotone in e, so with
+// G(u) = F + sum_{free, b_j >= u} q_j the largest pattern u* with G(u*) >= T is the pattern
+// of a free energy whose q is exactly v (G changes only where an element with q > 0 drops
+// out).  u* is found without a search over all the row's values:
+//   1. histogram: every free block with q > 0 adds q to the bin of its pattern, bins being
+//      half exponent levels counted down from the row's largest free pattern (b >> 22);
+//      q > 0 only within 53 levels of the row maximum, so 128 bins hold every such block.
+//      The sums are exact: q_j < 2^(52-c) with c = ceil(log2 nk) is split at bit 32-c into
+//      a low part (row total < 2^32) and a high part (row total < 2^30), each added with a
+//      32-bit shared-memory atomic.
+//   2. one warp scan of the 128 bins gives Q, T and the first bin k* (from the top) whose
+//      cumulative sum reaches T, so u* lies in bin k*, and A = G(top of bin k*) < T.
+//   3. the blocks of bin k* (usually a few: a factor-of-sqrt(2) band of energies) are
+//      moved to shared memory in index order, two per lane, and each computes G at its own
+//      pattern from the others; u* is the largest pattern with G >= T.
+//   4. if no block outside bin k* can have q == v (checked by quantizing the two patterns
+//      just outside the bin), the blocks above bin k* are kept, and the bin's own blocks
+//      are decided in shared memory (q > v kept, then ties in index order).
+// A row whose bin k* holds more than 64 blocks, or whose ties may cross the bin's edges,
+// takes the exact bisection over the bit patterns instead (at most 31 steps over all of the
+// row's elements).
 template <int MPL>
 __global__ void __launch_bounds__(kSelWarps * 32, MPL <= 8 ? 8 : (MPL <= 16 ? 6 : (MPL <= 20 ? 5 : 3)))
 select_mask_kernel(const __grid_constant__ SelectParams p) {
     static_assert(MPL >= 1 && MPL <= kSelMaxPerLane, "per-lane count");
-    __shared__ uint32_t cand_b[kSelWarps][kSelCompact];
-    __shared__ uint32_t cand_l[kSelWarps][kSelCompact];
-    __shared__ uint32_t cand_h[kSelWarps][kSelCompact];
+    constexpr int NB = kSelBins;
+    constexpr int BW = (MPL + 3) / 4;                        // words of packed bin bytes
+    __shared__ __align__(16) uint32_t hist_lo[kSelWarps][NB];
+    __shared__ __align__(16) uint32_t hist_hi[kSelWarps][NB];
+    __shared__ __align__(16) uint4 cand[kSelWarps][kSelCompact];   // (b, q low, q high, j)
+    __shared__ uint32_t kmask[kSelWarps][32];                      // kept candidates, by j
     const uint32_t wib = warp_id();
     const long long gw = static_cast<long long>(blockIdx.x) * kSelWarps + wib;
     if (gw >= static_cast<long long>(p.rows) * p.n_chunks) return;
@@ -115,6 +168,11 @@ select_mask_kernel(const __grid_constant__ SelectParams p) {
     auto join = [&](uint32_t hi_sum, uint32_t lo_sum) -> uint64_t {
         return (static_cast<uint64_t>(hi_sum) << cs) + lo_sum;
     };
+    uint32_t* hlo = hist_lo[wib];
+    uint32_t* hhi = hist_hi[wib];
+    reinterpret_cast<uint4*>(hlo)[lane] = make_uint4(0, 0, 0, 0);  // bins 4*lane .. 4*lane+3
+    reinterpret_cast<uint4*>(hhi)[lane] = make_uint4(0, 0, 0, 0);
+    __syncwarp();
 
     uint32_t fbits = 0;                                      // forced blocks of this row
     if (p.force) {
@@ -165,117 +223,200 @@ select_mask_kernel(const __grid_constant__ SelectParams p) {
             if (jd >= j0 && jd < j0 + MPL) kbits |= 1u << (jd - j0);
         } else {
             const int shift = 52 - float_exponent_p(xmax) - c;
-            uint32_t ql[MPL], qh[MPL];
-            uint32_t al = 0, ah = 0, fl = 0, fh = 0, bmax = 0;
+            // forced blocks: their q counts toward F; they are not free (pattern 0)
+            uint32_t fl = 0, fh = 0, bmax = 0;
+            if (__any_sync(0xffffffffu, fbits != 0u)) {
 #pragma unroll
-            for (int m = 0; m < MPL; ++m) {
-                const uint64_t q = quantize_bits(b[m], shift);
-                ql[m] = static_cast<uint32_t>(q) & lomask;
-                qh[m] = static_cast<uint32_t>(q >> cs);
-                al += ql[m];
-                ah += qh[m];
-                if ((fbits >> m) & 1u) {
-                    fl += ql[m];
-                    fh += qh[m];
-                    b[m] = 0u;                               // forced blocks are not free
+                for (int m = 0; m < MPL; ++m) {
+                    if ((fbits >> m) & 1u) {
+                        const uint64_t q = quantize_fast(b[m], shift);
+                        fl += static_cast<uint32_t>(q) & lomask;
+                        fh += static_cast<uint32_t>(q >> cs);
+                        b[m] = 0u;
+                    }
                 }
-                bmax = b[m] > bmax ? b[m] : bmax;
             }
-            const uint64_t Q = join(warp_sum_u32(ah), warp_sum_u32(al));
+#pragma unroll
+            for (int m = 0; m < MPL; ++m) bmax = b[m] > bmax ? b[m] : bmax;
             const uint64_t F = join(warp_sum_u32(fh), warp_sum_u32(fl));
             bmax = warp_max_u32(bmax);
-            uint64_t T = __double2ull_rz(ceil(__dmul_rn(p.tau[bi], __ull2double_rn(Q))));
-            if (T < 1) T = 1;
-            if (F < T) {
-                // G(u) over every free element of the row (u >= 1: forced and padding have b = 0)
-                auto G_all = [&](uint32_t u) -> uint64_t {
-                    uint32_t sl = 0, sh = 0;
+            const uint32_t btop = bmax >> 22;                 // bin 0: the top half level
+            // 1. histogram of the free blocks' q by half level below the top
+            uint32_t binw[BW];
 #pragma unroll
-                    for (int m = 0; m < MPL; ++m) {
-                        const bool in = b[m] >= u;
-                        sl += in ? ql[m] : 0u;
-                        sh += in ? qh[m] : 0u;
-                    }
-                    return F + join(warp_sum_u32(sh), warp_sum_u32(sl));
-                };
-                // 1. exponent level: G(0) = Q >= T, G((lvl(bmax)+1) << 23) = F < T
-                uint32_t lo = 0, hi = (bmax >> 23) + 1;
-                uint64_t A = F;                              // G(hi << 23)
-                while (hi - lo > 1) {
-                    const uint32_t mid = (lo + hi) >> 1;
-                    const uint64_t g = G_all(mid << 23);
-                    if (g >= T) lo = mid;
-                    else { hi = mid; A = g; }
-                }
-                const uint32_t lvl = lo;
-                // 2. low bits inside the level
-                uint32_t ul = lvl << 23, uh = (lvl + 1) << 23;
-                uint32_t cl = 0;
+            for (int w = 0; w < BW; ++w) binw[w] = 0xFFFFFFFFu;
+            bool far = false;
 #pragma unroll
-                for (int m = 0; m < MPL; ++m) cl += (b[m] != 0u && (b[m] >> 23) == lvl) ? 1u : 0u;
-                const uint32_t nc = warp_sum_u32(cl);
-                if (nc <= static_cast<uint32_t>(kSelCompact)) {
-                    uint32_t pos = warp_exclusive_scan(cl);
-#pragma unroll
-                    for (int m = 0; m < MPL; ++m) {
-                        if (b[m] != 0u && (b[m] >> 23) == lvl) {
-                            cand_b[wib][pos] = b[m];
-                            cand_l[wib][pos] = ql[m];
-                            cand_h[wib][pos] = qh[m];
-                            ++pos;
+            for (int m = 0; m < MPL; ++m) {
+                if (b[m] != 0u) {
+                    const uint64_t q = quantize_fast(b[m], shift);
+                    if (q != 0) {
+                        const uint32_t d = btop - (b[m] >> 22);
+                        if (d < static_cast<uint32_t>(NB)) {
+                            atomicAdd(hlo + d, static_cast<uint32_t>(q) & lomask);
+                            atomicAdd(hhi + d, static_cast<uint32_t>(q >> cs));
+                            binw[m >> 2] &= ~(0xFFu << (8 * (m & 3))) | (d << (8 * (m & 3)));
+                        } else {
+                            far = true;                      // cannot happen (q > 0 implies d <= 107)
                         }
                     }
+                }
+            }
+            __syncwarp();
+            // 2. scan of the bins (lane l: bins 4l .. 4l+3), clearing them for the next row
+            const uint4 lo4 = reinterpret_cast<const uint4*>(hlo)[lane];
+            const uint4 hi4 = reinterpret_cast<const uint4*>(hhi)[lane];
+            __syncwarp();
+            reinterpret_cast<uint4*>(hlo)[lane] = make_uint4(0, 0, 0, 0);
+            reinterpret_cast<uint4*>(hhi)[lane] = make_uint4(0, 0, 0, 0);
+            const uint64_t s0 = join(hi4.x, lo4.x), s1 = join(hi4.y, lo4.y), s2 = join(hi4.z, lo4.z),
+                           s3 = join(hi4.w, lo4.w);
+            const uint64_t p0 = s0, p1 = p0 + s1, p2 = p1 + s2, p3 = p2 + s3;   // inclusive, within lane
+            const uint64_t base = warp_exclusive_scan_u64(p3);
+            const uint64_t Qf = __shfl_sync(0xffffffffu, base + p3, 31);
+            const uint64_t Q = F + Qf;
+            uint64_t T = __double2ull_rz(ceil(__dmul_rn(p.tau[bi], __ull2double_rn(Q))));
+            if (T < 1) T = 1;
+            far = __any_sync(0xffffffffu, far);
+            if (F < T) {
+                // first bin whose cumulative sum reaches T
+                const uint64_t C = F + base;
+                const int kl = C + p0 >= T ? 0 : (C + p1 >= T ? 1 : (C + p2 >= T ? 2 : (C + p3 >= T ? 3 : 4)));
+                const uint32_t has = __ballot_sync(0xffffffffu, kl < 4);   // non-empty: the total reaches T
+                const int L = __ffs(has) - 1;
+                const int kls = __shfl_sync(0xffffffffu, kl, L);
+                const uint64_t Aown = C + (kl == 0 ? 0 : (kl == 1 ? p0 : (kl == 2 ? p1 : p2)));
+                const uint64_t A = __shfl_sync(0xffffffffu, Aown, L);        // G(top of bin k*)
+                const uint32_t kstar = static_cast<uint32_t>(4 * L + kls);
+                // 3. the blocks of bin k*, in index order
+                uint32_t cmask = 0;                          // this lane's blocks in bin k*
+#pragma unroll
+                for (int m = 0; m < MPL; ++m)
+                    cmask |= (((binw[m >> 2] >> (8 * (m & 3))) & 0xFFu) == kstar ? 1u : 0u) << m;
+                const uint32_t cl = __popc(cmask);
+                const uint32_t nc = warp_sum_u32(cl);
+                bool done = false;
+                if (!far && nc <= static_cast<uint32_t>(kSelCompact)) {
+                    const uint32_t pos0 = warp_exclusive_scan(cl);
+                    uint4* cw = cand[wib];
+                    // each block's slot is fixed by the blocks before it (so the slots are in
+                    // index order); its q is filled in by the lane that reads the slot
+#pragma unroll
+                    for (int m = 0; m < MPL; ++m)
+                        if ((cmask >> m) & 1u)
+                            cw[pos0 + __popc(cmask & ((1u << m) - 1u))] =
+                                make_uint4(b[m], 0u, 0u, static_cast<uint32_t>(j0 + m));
+                    kmask[wib][lane] = 0u;
                     __syncwarp();
                     const bool v0 = lane < nc, v1 = lane + 32 < nc;
-                    const uint32_t b0 = v0 ? cand_b[wib][lane] : 0u, b1 = v1 ? cand_b[wib][lane + 32] : 0u;
-                    const uint32_t l0 = v0 ? cand_l[wib][lane] : 0u, l1 = v1 ? cand_l[wib][lane + 32] : 0u;
-                    const uint32_t h0 = v0 ? cand_h[wib][lane] : 0u, h1 = v1 ? cand_h[wib][lane + 32] : 0u;
-                    __syncwarp();
-                    // G(u) = A + (level elements with b >= u), for u inside the level
-                    while (uh - ul > 1) {
-                        const uint32_t mid = ul + ((uh - ul) >> 1);
-                        const uint32_t sl = (b0 >= mid ? l0 : 0u) + (b1 >= mid ? l1 : 0u);
-                        const uint32_t sh = (b0 >= mid ? h0 : 0u) + (b1 >= mid ? h1 : 0u);
-                        if (A + join(warp_sum_u32(sh), warp_sum_u32(sl)) >= T) ul = mid;
-                        else uh = mid;
+                    uint4 c0 = v0 ? cw[lane] : make_uint4(0, 0, 0, 0);
+                    uint4 c1 = v1 ? cw[lane + 32] : make_uint4(0, 0, 0, 0);
+                    if (v0) {
+                        const uint64_t q = quantize_fast(c0.x, shift);
+                        c0.y = static_cast<uint32_t>(q);
+                        c0.z = static_cast<uint32_t>(q >> 32);
+                        cw[lane] = c0;
                     }
-                } else {
+                    if (v1) {
+                        const uint64_t q = quantize_fast(c1.x, shift);
+                        c1.y = static_cast<uint32_t>(q);
+                        c1.z = static_cast<uint32_t>(q >> 32);
+                        cw[lane + 32] = c1;
+                    }
+                    __syncwarp();
+                    // G at each candidate's own pattern
+                    uint64_t G0 = A, G1 = A;
+                    for (uint32_t x = 0; x < nc; ++x) {
+                        const uint4 e = cw[x];
+                        const uint64_t qe = (static_cast<uint64_t>(e.z) << 32) | e.y;
+                        if (e.x >= c0.x) G0 += qe;
+                        if (nc > 32 && e.x >= c1.x) G1 += qe;
+                    }
+                    const uint32_t ustar =
+                        warp_max_u32(max((v0 && G0 >= T) ? c0.x : 0u, (v1 && G1 >= T) ? c1.x : 0u));
+                    const uint64_t v = quantize_fast(ustar, shift);       // > 0 (see above)
+                    // 4. no block outside bin k* may tie with v
+                    const uint32_t top = btop - kstar;
+                    const uint32_t lo_p = top << 22, hi_p = (top + 1) << 22;
+                    const bool straddle = (lo_p > 0 && quantize_fast(lo_p - 1, shift) == v) ||
+                                          quantize_fast(hi_p, shift) == v;
+                    if (!straddle && v != 0) {
+                        const uint64_t q0 = (static_cast<uint64_t>(c0.z) << 32) | c0.y;
+                        const uint64_t q1 = (static_cast<uint64_t>(c1.z) << 32) | c1.y;
+                        const bool gt0 = v0 && q0 > v, gt1 = v1 && q1 > v;
+                        const bool eq0 = v0 && q0 == v, eq1 = v1 && q1 == v;
+                        const uint64_t R = T - A - warp_sum_u64((gt0 ? q0 : 0ull) + (gt1 ? q1 : 0ull));   // > 0
+                        // exact ceil(R / v): a float estimate, then integer steps (R <= nk * v)
+                        uint64_t need = static_cast<uint64_t>(__fdividef(__ull2float_rn(R), __ull2float_rn(v)));
+                        while (need * v < R) ++need;
+                        while (need > 0 && (need - 1) * v >= R) --need;
+                        const uint32_t e0 = __ballot_sync(0xffffffffu, eq0), e1 = __ballot_sync(0xffffffffu, eq1);
+                        const uint32_t r0 = __popc(e0 & lanemask_lt()), r1 = __popc(e0) + __popc(e1 & lanemask_lt());
+                        if (gt0 || (eq0 && r0 < need)) atomicOr(&kmask[wib][c0.w >> 5], 1u << (c0.w & 31));
+                        if (gt1 || (eq1 && r1 < need)) atomicOr(&kmask[wib][c1.w >> 5], 1u << (c1.w & 31));
+                        __syncwarp();
+#pragma unroll
+                        for (int m = 0; m < MPL; ++m) {
+                            const uint32_t d = (binw[m >> 2] >> (8 * (m & 3))) & 0xFFu;
+                            const int j = j0 + m;
+                            const bool k = d < kstar || (d == kstar && ((kmask[wib][j >> 5] >> (j & 31)) & 1u));
+                            kbits |= (k ? 1u : 0u) << m;
+                        }
+                        done = true;
+                    }
+                    __syncwarp();                                 // candidates read before reuse
+                }
+                if (!done) {
+                    // exact bisection over the bit patterns (rare rows); q is recomputed from
+                    // the patterns, so this path adds no per-block registers to the fast path
+                    auto G_all = [&](uint32_t u) -> uint64_t {   // u >= 1: forced and padding have b = 0
+                        uint32_t sl = 0, sh = 0;
+                        const int sh2 = opaque(shift);
+#pragma unroll
+                        for (int m = 0; m < MPL; ++m) {
+                            if (b[m] >= u) {
+                                const uint64_t q = quantize_bits(b[m], sh2);
+                                sl += static_cast<uint32_t>(q) & lomask;
+                                sh += static_cast<uint32_t>(q >> cs);
+                            }
+                        }
+                        return F + join(warp_sum_u32(sh), warp_sum_u32(sl));
+                    };
+                    uint32_t ul = 0, uh = bmax + 1;              // G(0) = Q >= T, G(bmax + 1) = F < T
                     while (uh - ul > 1) {
                         const uint32_t mid = ul + ((uh - ul) >> 1);
                         if (G_all(mid) >= T) ul = mid;
                         else uh = mid;
                     }
-                }
-                const uint64_t v = quantize_bits(ul, shift);    // > 0 (see above)
-                // free blocks above v are kept; ties at v are taken in index order
-                uint32_t gl = 0, gh = 0, ce = 0;
-                uint32_t eqbits = 0;
+                    const uint64_t v = quantize_bits(ul, shift);
+                    uint32_t gl = 0, gh = 0, ce = 0, eqbits = 0;
+                    const int sh3 = opaque(shift);
 #pragma unroll
-                for (int m = 0; m < MPL; ++m) {
-                    const uint64_t q = (static_cast<uint64_t>(qh[m]) << cs) | ql[m];
-                    const bool fr = !((fbits >> m) & 1u) && j0 + m < nk;
-                    if (fr && q > v) {
-                        kbits |= 1u << m;
-                        gl += ql[m];
-                        gh += qh[m];
-                    } else if (fr && q == v) {
-                        eqbits |= 1u << m;
-                        ++ce;
+                    for (int m = 0; m < MPL; ++m) {
+                        const uint64_t q = b[m] ? quantize_bits(b[m], sh3) : 0ull;   // forced: b = 0
+                        if (q > v) {
+                            kbits |= 1u << m;
+                            gl += static_cast<uint32_t>(q) & lomask;
+                            gh += static_cast<uint32_t>(q >> cs);
+                        } else if (q == v) {
+                            eqbits |= 1u << m;
+                            ++ce;
+                        }
                     }
-                }
-                const uint64_t R = T - F - join(warp_sum_u32(gh), warp_sum_u32(gl));   // > 0
-                uint64_t need = v ? static_cast<uint64_t>(ceil(__ddiv_rn(__ull2double_rn(R), __ull2double_rn(v))))
-                                  : 0ull;
-                if (v) {
-                    while (need * v < R) ++need;                   // exact ceil(R / v)
-                    while (need > 0 && (need - 1) * v >= R) --need;
-                }
-                uint64_t rank = warp_exclusive_scan(ce);
+                    const uint64_t R = T - F - join(warp_sum_u32(gh), warp_sum_u32(gl));   // > 0
+                    uint64_t need =
+                        v ? static_cast<uint64_t>(ceil(__ddiv_rn(__ull2double_rn(R), __ull2double_rn(v)))) : 0ull;
+                    if (v) {
+                        while (need * v < R) ++need;
+                        while (need > 0 && (need - 1) * v >= R) --need;
+                    }
+                    uint64_t rank = warp_exclusive_scan(ce);
 #pragma unroll
-                for (int m = 0; m < MPL; ++m) {
-                    if ((eqbits >> m) & 1u) {
-                        if (rank < need) kbits |= 1u << m;
-                        ++rank;
+                    for (int m = 0; m < MPL; ++m) {
+                        if ((eqbits >> m) & 1u) {
+                            if (rank < need) kbits |= 1u << m;
+                            ++rank;
+                        }
                     }
                 }
             }
