@@ -106,11 +106,22 @@ __device__ __forceinline__ uint64_t warp_exclusive_scan_u64(uint64_t v) {
 // take the integer path.  Same value as quantize_bits, in a handful of instructions.
 __device__ __forceinline__ uint64_t quantize_fast(uint32_t x, int shift) {
     const uint32_t E = x >> 23;
-    if (E == 0u) return quantize_bits(x, shift);
     const uint32_t hi = ((E + 896u + static_cast<uint32_t>(shift)) << 20) | ((x & 0x7FFFFFu) >> 3);
-    const double d = __hiloint2double(static_cast<int>(hi), static_cast<int>(x << 29));
-    const double r = __dadd_rn(d, 4503599627370496.0);           // + 2^52
+    const double dn = __hiloint2double(static_cast<int>(hi), static_cast<int>(x << 29));
+    // a subnormal x is its significand times 2^-149: an exact integer conversion and an exact
+    // scaling by a power of two (built from its exponent field)
+    const double ds = __dmul_rn(__uint2double_rn(x & 0x7FFFFFu),
+                                __hiloint2double(static_cast<int>((874u + static_cast<uint32_t>(shift)) << 20), 0));
+    const double r = __dadd_rn(E ? dn : ds, 4503599627370496.0);  // + 2^52
     return static_cast<uint64_t>(__double_as_longlong(r)) & 0xFFFFFFFFFFFFFull;
+}
+
+// Shared-memory reductions by shared-space address (no generic-address check).
+__device__ __forceinline__ void red_shared_add(uint32_t addr, uint32_t v) {
+    asm volatile("red.shared.add.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+__device__ __forceinline__ void red_shared_or(uint32_t addr, uint32_t v) {
+    asm volatile("red.shared.or.b32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
 }
 
 // Minimal tau-energy selection, one warp per (row, chunk of batch entries); lane l holds
@@ -146,7 +157,6 @@ __global__ void __launch_bounds__(kSelWarps * 32, MPL <= 8 ? 8 : (MPL <= 16 ? 6 
 select_mask_kernel(const __grid_constant__ SelectParams p) {
     static_assert(MPL >= 1 && MPL <= kSelMaxPerLane, "per-lane count");
     constexpr int NB = kSelBins;
-    constexpr int BW = (MPL + 3) / 4;                        // words of packed bin bytes
     __shared__ __align__(16) uint32_t hist_lo[kSelWarps][NB];
     __shared__ __align__(16) uint32_t hist_hi[kSelWarps][NB];
     __shared__ __align__(16) uint4 cand[kSelWarps][kSelCompact];   // (b, q low, q high, j)
@@ -242,10 +252,11 @@ select_mask_kernel(const __grid_constant__ SelectParams p) {
             bmax = warp_max_u32(bmax);
             const uint32_t btop = bmax >> 22;                 // bin 0: the top half level
             // 1. histogram of the free blocks' q by half level below the top
-            uint32_t binw[BW];
+            uint32_t dm[MPL];                                 // bin of each block, 0xFF: none
 #pragma unroll
-            for (int w = 0; w < BW; ++w) binw[w] = 0xFFFFFFFFu;
+            for (int m = 0; m < MPL; ++m) dm[m] = 0xFFu;
             bool far = false;
+            const uint32_t hlo_a = smem_u32(hlo), hhi_a = smem_u32(hhi);
 #pragma unroll
             for (int m = 0; m < MPL; ++m) {
                 if (b[m] != 0u) {
@@ -253,9 +264,9 @@ select_mask_kernel(const __grid_constant__ SelectParams p) {
                     if (q != 0) {
                         const uint32_t d = btop - (b[m] >> 22);
                         if (d < static_cast<uint32_t>(NB)) {
-                            atomicAdd(hlo + d, static_cast<uint32_t>(q) & lomask);
-                            atomicAdd(hhi + d, static_cast<uint32_t>(q >> cs));
-                            binw[m >> 2] &= ~(0xFFu << (8 * (m & 3))) | (d << (8 * (m & 3)));
+                            red_shared_add(hlo_a + 4 * d, static_cast<uint32_t>(q) & lomask);
+                            red_shared_add(hhi_a + 4 * d, static_cast<uint32_t>(q >> cs));
+                            dm[m] = d;
                         } else {
                             far = true;                      // cannot happen (q > 0 implies d <= 107)
                         }
@@ -292,7 +303,7 @@ select_mask_kernel(const __grid_constant__ SelectParams p) {
                 uint32_t cmask = 0;                          // this lane's blocks in bin k*
 #pragma unroll
                 for (int m = 0; m < MPL; ++m)
-                    cmask |= (((binw[m >> 2] >> (8 * (m & 3))) & 0xFFu) == kstar ? 1u : 0u) << m;
+                    cmask |= (dm[m] == kstar ? 1u : 0u) << m;
                 const uint32_t cl = __popc(cmask);
                 const uint32_t nc = warp_sum_u32(cl);
                 bool done = false;
@@ -352,12 +363,13 @@ select_mask_kernel(const __grid_constant__ SelectParams p) {
                         while (need > 0 && (need - 1) * v >= R) --need;
                         const uint32_t e0 = __ballot_sync(0xffffffffu, eq0), e1 = __ballot_sync(0xffffffffu, eq1);
                         const uint32_t r0 = __popc(e0 & lanemask_lt()), r1 = __popc(e0) + __popc(e1 & lanemask_lt());
-                        if (gt0 || (eq0 && r0 < need)) atomicOr(&kmask[wib][c0.w >> 5], 1u << (c0.w & 31));
-                        if (gt1 || (eq1 && r1 < need)) atomicOr(&kmask[wib][c1.w >> 5], 1u << (c1.w & 31));
+                        const uint32_t km_a = smem_u32(kmask[wib]);
+                        if (gt0 || (eq0 && r0 < need)) red_shared_or(km_a + 4 * (c0.w >> 5), 1u << (c0.w & 31));
+                        if (gt1 || (eq1 && r1 < need)) red_shared_or(km_a + 4 * (c1.w >> 5), 1u << (c1.w & 31));
                         __syncwarp();
 #pragma unroll
                         for (int m = 0; m < MPL; ++m) {
-                            const uint32_t d = (binw[m >> 2] >> (8 * (m & 3))) & 0xFFu;
+                            const uint32_t d = dm[m];
                             const int j = j0 + m;
                             const bool k = d < kstar || (d == kstar && ((kmask[wib][j >> 5] >> (j & 31)) & 1u));
                             kbits |= (k ? 1u : 0u) << m;
@@ -441,8 +453,10 @@ select_mask_kernel(const __grid_constant__ SelectParams p) {
                     if (j0 + m < nk) M[j0 + m] = static_cast<uint8_t>((kbits >> m) & 1u);
             }
         }
+        if (p.count_accum) {
 #pragma unroll
-        for (int m = 0; m < MPL; ++m) cnt[m >> 2] += ((kbits >> m) & 1u) << (8 * (m & 3));
+            for (int m = 0; m < MPL; ++m) cnt[m >> 2] += ((kbits >> m) & 1u) << (8 * (m & 3));
+        }
     }
     if (p.count_accum) {
 #pragma unroll
