@@ -15,11 +15,15 @@ def pytest_configure(config):
 
 
 def pytest_sessionstart(session):
-    """A fresh checkout has no libcalibatt.so (built files are not versioned): build it
-    in-tree once, with nvcc for sm_100a, before the tests load it."""
+    """Build libcalibatt.so in-tree (nvcc, sm_100a) before the tests load it: a fresh
+    checkout has none, and a library older than its sources would test old code.  The
+    build skips itself when the library is up to date.  Without nvcc the oracle and format
+    tests still run; the tests that load the library then report it missing."""
     from calibrated_block_sparse_calib_b200 import build
-    if not os.path.exists(build.LIB):
+    try:
         build.build()
+    except RuntimeError as e:
+        sys.stderr.write(f"libcalibatt.so not built: {e}\n")
 
 
 def to64(t):
