@@ -446,6 +446,70 @@ def test_attention_empty_rows_write_zero():
     check_attn(O, O_ref)
 
 
+def test_persistent_work_order_and_subsets():
+    """The attention CTAs take work items by cancelling not-yet-started CTAs, so the set of
+    items processed is exactly the work list, whatever its order: a random permutation of
+    the schedule gives bitwise the same output (each item's arithmetic does not depend on
+    the order), a list without some rows leaves those rows untouched, and repeated calls
+    on the same list agree."""
+    wl = _shape(3, 128, 6, 10, 23, 128)
+    q, k, v = _inputs(wl, seed=77)
+    nb = wl.shape.nblk
+    rng = np.random.default_rng(12)
+    m = _rand_mask(rng, 3, nb, nb, 0.3)
+    m[1, 2] = 0                                                    # an empty row
+    bl = _blist(m, 128)
+    ref, lse_ref = ops.sparse_attn_fwd(q, k, v, bl, return_lse=True)
+    O_ref, _ = oracle.sparse_attention(to64(q), to64(k), to64(v), 1 / math.sqrt(128), 128, m)
+    check_attn(ref, O_ref)
+    for trial in range(3):
+        perm = torch.from_numpy(rng.permutation(bl.work.cpu().numpy()).astype(np.int32)).cuda()
+        blp = ops.BlockList(bl.H, bl.nq, bl.nk, bl.block, bl.row_ptr, bl.col_idx, perm)
+        o, l = ops.sparse_attn_fwd(q, k, v, blp, return_lse=True)
+        assert torch.equal(o, ref) and torch.equal(l, lse_ref), trial
+    # a subset of the items: the rows left out keep what the output held before
+    keep = rng.random(bl.work.numel()) < 0.6
+    sub = bl.work[torch.from_numpy(keep).cuda()].contiguous()
+    bls = ops.BlockList(bl.H, bl.nq, bl.nk, bl.block, bl.row_ptr, bl.col_idx, sub)
+    out = torch.full_like(ref, 7.0)
+    ops.sparse_attn_fwd(q, k, v, bls, out=out)
+    ops.device_check()
+    rows = torch.zeros(3, wl.shape.N, dtype=torch.bool)
+    for item in sub.cpu().tolist():
+        h, i = item >> 16, item & 0xFFFF
+        rows[h, i * 128:(i + 1) * 128] = True
+    o, r = out.cpu(), ref.cpu()
+    assert torch.equal(o[rows], r[rows])
+    assert torch.all(o[~rows] == 7.0)
+
+
+@pytest.mark.parametrize("n_items", [1, 147, 148, 149, 300])
+def test_persistent_grid_sizes_around_the_sm_count(n_items):
+    """Work lists shorter than, equal to and just above the 148 SMs (the first items run on
+    their own CTAs, the rest are taken by cancellation) against the oracle."""
+    wl = _shape(4, 64, 8, 16, 40, 64)                              # 5120 tokens, 80 blocks
+    q, k, v = _inputs(wl, seed=n_items)
+    nb = wl.shape.nblk
+    rng = np.random.default_rng(n_items)
+    m = _rand_mask(rng, 4, nb, nb, 0.2)
+    bl = _blist(m, 64)
+    work = bl.work[:n_items].contiguous()
+    blw = ops.BlockList(bl.H, bl.nq, bl.nk, bl.block, bl.row_ptr, bl.col_idx, work)
+    out = torch.zeros_like(q)
+    ops.sparse_attn_fwd(q, k, v, blw, out=out)
+    ops.device_check()
+    items = work.cpu().tolist()
+    heads = sorted({it >> 16 for it in items})
+    O_ref, _ = oracle.sparse_attention(to64(q[heads]), to64(k[heads]), to64(v[heads]), 1 / 8.0, 64, m[heads])
+    o = to64(out)
+    for it in items:
+        h, i = it >> 16, it & 0xFFFF
+        sl = slice(i * 64, min((i + 1) * 64, wl.shape.N))
+        ref_rows = O_ref[heads.index(h), sl]
+        d = np.abs(o[h, sl] - ref_rows)
+        assert float((d - (ATTN_MAXABS + half_ulp_bf16(ref_rows))).max()) <= 0, (h, i)
+
+
 @pytest.mark.parametrize("with_lse", [False, True])
 def test_masked_blocks_do_not_matter_bitwise(with_lse):
     # Rows keeping 0..4 blocks (one row empty): outputs are bit-identical across repeated
