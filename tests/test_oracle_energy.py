@@ -101,6 +101,20 @@ def test_energy_mean_single_input_identity():
     np.testing.assert_allclose(m, (2 * e.astype(np.float64)).astype(np.float32), rtol=0)
 
 
+def test_energy_mean_rows_sum_to_one_softmax_row_per_query():
+    """Each input's query rows sum to one softmax row each (sum_j E[i, j] = |I_i|), so the
+    mean over inputs keeps that sum; the plain sum over three inputs (the 1/D_cal factor
+    dropped) would give 3 |I_i| and fails this pin."""
+    Es = []
+    for seed in (11, 12, 13):
+        q, k = _rand(1, 200, 8, seed)
+        Es.append(oracle.block_energy(q, k, 0.7, 64))
+    rows = np.array([64, 64, 64, 8], np.float64)
+    mean = oracle.energy_mean(Es).astype(np.float64)
+    np.testing.assert_allclose(mean.sum(axis=2)[0], rows, rtol=1e-6)
+    assert not np.allclose(sum(Es).sum(axis=2)[0], rows, rtol=1e-3)
+
+
 def test_row_sum_pin_catches_a_mean_instead_of_a_sum(monkeypatch):
     # Plant a plausible mistake in the oracle (block mean instead of block sum) and
     # check the row-sum pin fails: the pins discriminate.
