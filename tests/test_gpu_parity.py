@@ -203,6 +203,32 @@ def test_select_batched_many_entries_split_over_warps():
         np.testing.assert_array_equal(masks[b], oracle.select_mask(e[b], taus[b]))
 
 
+@pytest.mark.parametrize("workload,nb", [("wan13b", 32), ("wan14b720p", 2)])
+def test_select_batched_full_size_sampled_rows(workload, nb):
+    """The selection launch bench.py times, at full size: nb distinct energy matrices of the
+    workload's shape (the GPU energy pass on its inputs, each entry rescaled per row by a
+    seeded factor), tau(t) = 0.99 / 0.95 / 0.9 over the entries.  Sampled (entry, row) pairs
+    are bit-exact against the oracle's selection of the same energies."""
+    wl = synth.WORKLOADS[workload]
+    s = wl.shape
+    q, k, _ = synth.make_qkv(wl, device="cuda")
+    E = ops.block_energy(q, k, s.block)
+    del q, k
+    g = torch.Generator(device="cuda")
+    g.manual_seed(5)
+    batch = torch.stack([E * (0.5 + torch.rand(E.shape[:2] + (1,), generator=g, device="cuda"))
+                         for _ in range(nb)]).contiguous()
+    taus = [0.99 if b < nb * 3 // 8 else (0.95 if b < nb * 6 // 8 else 0.9) for b in range(nb)]
+    got = ops.select_mask_batched(batch, taus)
+    ops.device_check()
+    rng = np.random.default_rng(9)
+    for _ in range(120):
+        b, h, i = int(rng.integers(nb)), int(rng.integers(s.H)), int(rng.integers(s.nblk))
+        e = batch[b, h, i].cpu().numpy()
+        ref = oracle.select_row(e, taus[b], i).astype(np.uint8)
+        np.testing.assert_array_equal(got[b, h, i].cpu().numpy(), ref, err_msg=f"entry {b} head {h} row {i}")
+
+
 @pytest.mark.parametrize("n_inputs,rho", [(1, (1, 2)), (3, (1, 2)), (4, (1, 2)), (5, (1, 3)), (4, (0, 1))])
 def test_aggregate_bit_exact(n_inputs, rho):
     rng = np.random.default_rng(n_inputs * 7 + rho[0])
