@@ -161,6 +161,7 @@ select_mask_kernel(const __grid_constant__ SelectParams p) {
     __shared__ __align__(16) uint32_t hist_hi[kSelWarps][NB];
     __shared__ __align__(16) uint4 cand[kSelWarps][kSelCompact];   // (b, q low, q high, j)
     __shared__ uint32_t kmask[kSelWarps][32];                      // kept candidates, by j
+    __shared__ uint32_t rowb[kSelWarps][32 * MPL];                 // the row's patterns (fallback)
     const uint32_t wib = warp_id();
     const long long gw = static_cast<long long>(blockIdx.x) * kSelWarps + wib;
     if (gw >= static_cast<long long>(p.rows) * p.n_chunks) return;
@@ -379,15 +380,20 @@ select_mask_kernel(const __grid_constant__ SelectParams p) {
                     __syncwarp();                                 // candidates read before reuse
                 }
                 if (!done) {
-                    // exact bisection over the bit patterns (rare rows); q is recomputed from
-                    // the patterns, so this path adds no per-block registers to the fast path
+                    // exact bisection over the bit patterns (rare rows).  The row's free
+                    // patterns go to shared memory and the loops below run over it without
+                    // unrolling, so this path stays small next to the fast one.
+                    uint32_t* rb = rowb[wib];
+#pragma unroll
+                    for (int m = 0; m < MPL; ++m) rb[j0 + m] = b[m];
+                    __syncwarp();
                     auto G_all = [&](uint32_t u) -> uint64_t {   // u >= 1: forced and padding have b = 0
                         uint32_t sl = 0, sh = 0;
-                        const int sh2 = opaque(shift);
-#pragma unroll
-                        for (int m = 0; m < MPL; ++m) {
-                            if (b[m] >= u) {
-                                const uint64_t q = quantize_bits(b[m], sh2);
+#pragma unroll 1
+                        for (int x = static_cast<int>(lane); x < 32 * MPL; x += 32) {
+                            const uint32_t bx = rb[x];
+                            if (bx >= u) {
+                                const uint64_t q = quantize_fast(bx, shift);
                                 sl += static_cast<uint32_t>(q) & lomask;
                                 sh += static_cast<uint32_t>(q >> cs);
                             }
@@ -400,12 +406,14 @@ select_mask_kernel(const __grid_constant__ SelectParams p) {
                         if (G_all(mid) >= T) ul = mid;
                         else uh = mid;
                     }
-                    const uint64_t v = quantize_bits(ul, shift);
+                    const uint64_t v = quantize_fast(ul, shift);
+                    // free blocks above v are kept; ties at v in index order (this lane's
+                    // blocks are j0 .. j0 + MPL - 1)
                     uint32_t gl = 0, gh = 0, ce = 0, eqbits = 0;
-                    const int sh3 = opaque(shift);
-#pragma unroll
+#pragma unroll 1
                     for (int m = 0; m < MPL; ++m) {
-                        const uint64_t q = b[m] ? quantize_bits(b[m], sh3) : 0ull;   // forced: b = 0
+                        const uint32_t bx = rb[j0 + m];              // forced and padding: 0
+                        const uint64_t q = bx ? quantize_fast(bx, shift) : 0ull;
                         if (q > v) {
                             kbits |= 1u << m;
                             gl += static_cast<uint32_t>(q) & lomask;
@@ -416,20 +424,21 @@ select_mask_kernel(const __grid_constant__ SelectParams p) {
                         }
                     }
                     const uint64_t R = T - F - join(warp_sum_u32(gh), warp_sum_u32(gl));   // > 0
-                    uint64_t need =
-                        v ? static_cast<uint64_t>(ceil(__ddiv_rn(__ull2double_rn(R), __ull2double_rn(v)))) : 0ull;
+                    // exact ceil(R / v): a float estimate, then integer steps (R <= nk * v)
+                    uint64_t need = v ? static_cast<uint64_t>(__fdividef(__ull2float_rn(R), __ull2float_rn(v))) : 0ull;
                     if (v) {
                         while (need * v < R) ++need;
                         while (need > 0 && (need - 1) * v >= R) --need;
                     }
                     uint64_t rank = warp_exclusive_scan(ce);
-#pragma unroll
+#pragma unroll 1
                     for (int m = 0; m < MPL; ++m) {
                         if ((eqbits >> m) & 1u) {
                             if (rank < need) kbits |= 1u << m;
                             ++rank;
                         }
                     }
+                    __syncwarp();                                 // rb read before the next entry
                 }
             }
         }
