@@ -670,6 +670,28 @@ def test_wan13b_sampled_blocks(out_dtype):
     check_attn(O[heads], O_ref, rows=rows)
 
 
+@pytest.mark.parametrize("density", [0.10, 1.0])
+def test_wan13b_density_sweep_sampled_blocks(density):
+    """The density sweep's launches at full size: the 10% generator mask (many short items
+    per persistent CTA) and the all-kept list (this build's dense kernel), sampled query
+    blocks of three heads against the oracle, with the LSE."""
+    wl = synth.WORKLOADS["wan13b"]
+    s = wl.shape
+    q, k, v = synth.make_qkv(wl, device="cuda")
+    mask = (synth.make_head_masks(wl, density=density) if density < 1
+            else np.ones((s.H, s.nblk, s.nblk), np.uint8))
+    O, L = ops.sparse_attn_fwd(q, k, v, _blist(mask, s.block), return_lse=True)
+    ops.device_check()
+    rng = np.random.default_rng(int(density * 100))
+    blocks = sorted(set(rng.choice(s.nblk - 1, size=5, replace=False).tolist()) | {s.nblk - 1})
+    rows = np.concatenate([np.arange(i * s.block, min((i + 1) * s.block, s.N)) for i in blocks])
+    heads = [1, 7]
+    qh, kh, vh = (to64(t[heads]) for t in (q, k, v))
+    O_ref, L_ref = oracle.sparse_attention(qh, kh, vh, 1 / math.sqrt(s.D), s.block, mask[heads], q_blocks=blocks)
+    check_attn(O[heads], O_ref, rows=rows)
+    np.testing.assert_allclose(to64(L[heads])[:, rows], L_ref[:, rows], atol=5e-4, rtol=0)
+
+
 def test_wait_timeout_selftest_keeps_context_usable(tiny_inputs):
     assert ops.selftest_wait_timeout(2000) == ops.CALIB_ERR_TIMEOUT
     ops.device_check()                                   # the status word was cleared
