@@ -54,33 +54,6 @@ __device__ __forceinline__ int float_exponent_p(uint32_t bits) {
     return msb - 148;
 }
 
-// q = rint(e * 2^shift), ties to even, for e >= 0 given by its binary32 bits x.  The
-// significand m and exponent give e = m * 2^(E' - 150) (E' = max(E, 1)), so q = m * 2^k
-// with k = E' - 150 + shift: a left shift when k >= 0, else a right shift by s = -k with
-// round-half-even on the bits shifted out.  This is the same integer that rounding the
-// (exact) binary64 product e * 2^shift gives.
-__device__ __forceinline__ uint64_t quantize_bits(uint32_t x, int shift) {
-    const uint32_t E = x >> 23;
-    const uint32_t m = E ? ((x & 0x7FFFFFu) | 0x800000u) : (x & 0x7FFFFFu);
-    const int k = static_cast<int>(E ? E : 1u) - 150 + shift;
-    if (k >= 0) return static_cast<uint64_t>(m) << k;
-    const int s = -k;
-    if (s >= 32) return 0;
-    const uint32_t qt = m >> s;
-    const uint32_t rem = m & ((1u << s) - 1u);
-    const uint32_t half = 1u << (s - 1);
-    return qt + ((rem > half || (rem == half && (qt & 1u))) ? 1u : 0u);
-}
-
-// A copy of x that the compiler cannot see through: a value recomputed from it is not
-// merged with (or hoisted to) an earlier computation, so no per-block results stay live
-// across a loop just to be reused.
-__device__ __forceinline__ int opaque(int x) {
-    int y;
-    asm volatile("mov.b32 %0, %1;" : "=r"(y) : "r"(x));
-    return y;
-}
-
 // 64-bit sum over the lanes of a warp (butterfly of 32-bit shuffles).
 __device__ __forceinline__ uint64_t warp_sum_u64(uint64_t v) {
 #pragma unroll
@@ -99,12 +72,16 @@ __device__ __forceinline__ uint64_t warp_exclusive_scan_u64(uint64_t v) {
     return x - v;
 }
 
-// quantize_bits on the FP64 pipe: for a normal binary32 x (exponent field E >= 1) the
-// binary64 with exponent E + 896 + shift and x's significand is exactly e * 2^shift (no
-// overflow or underflow for shift in [-86, 200]); adding 2^52 rounds it to an integer, half
-// to even (e * 2^shift < 2^52 here), which is then the low 52 bits of the sum.  Subnormal x
-// take the integer path.  Same value as quantize_bits, in a handful of instructions.
-__device__ __forceinline__ uint64_t quantize_fast(uint32_t x, int shift) {
+// q = rint(e * 2^shift), ties to even, for e >= 0 given by its binary32 bits x, computed
+// on the FP64 pipe.  For a normal x (exponent field E >= 1) the binary64 with exponent
+// E + 896 + shift and x's significand is exactly e * 2^shift (no overflow or underflow for
+// shift in [-86, 200]).  A subnormal x is its significand times 2^-149: an exact integer
+// conversion scaled by an exact power of two.  Adding 2^52 then rounds the product to an
+// integer, half to even (e * 2^shift < 2^52 here), and q is the low 52 bits of the sum.
+// This is the same integer as rounding the significand shifted by E' - 150 + shift bits
+// (E' = max(E, 1)) with round-half-even on the bits shifted out; a CPU check compared the
+// two on every exponent and on exact halves.
+__device__ __forceinline__ uint64_t quantize_energy(uint32_t x, int shift) {
     const uint32_t E = x >> 23;
     const uint32_t hi = ((E + 896u + static_cast<uint32_t>(shift)) << 20) | ((x & 0x7FFFFFu) >> 3);
     const double dn = __hiloint2double(static_cast<int>(hi), static_cast<int>(x << 29));
@@ -240,7 +217,7 @@ select_mask_kernel(const __grid_constant__ SelectParams p) {
 #pragma unroll
                 for (int m = 0; m < MPL; ++m) {
                     if ((fbits >> m) & 1u) {
-                        const uint64_t q = quantize_fast(b[m], shift);
+                        const uint64_t q = quantize_energy(b[m], shift);
                         fl += static_cast<uint32_t>(q) & lomask;
                         fh += static_cast<uint32_t>(q >> cs);
                         b[m] = 0u;
@@ -261,7 +238,7 @@ select_mask_kernel(const __grid_constant__ SelectParams p) {
 #pragma unroll
             for (int m = 0; m < MPL; ++m) {
                 if (b[m] != 0u) {
-                    const uint64_t q = quantize_fast(b[m], shift);
+                    const uint64_t q = quantize_energy(b[m], shift);
                     if (q != 0) {
                         const uint32_t d = btop - (b[m] >> 22);
                         if (d < static_cast<uint32_t>(NB)) {
@@ -324,13 +301,13 @@ select_mask_kernel(const __grid_constant__ SelectParams p) {
                     uint4 c0 = v0 ? cw[lane] : make_uint4(0, 0, 0, 0);
                     uint4 c1 = v1 ? cw[lane + 32] : make_uint4(0, 0, 0, 0);
                     if (v0) {
-                        const uint64_t q = quantize_fast(c0.x, shift);
+                        const uint64_t q = quantize_energy(c0.x, shift);
                         c0.y = static_cast<uint32_t>(q);
                         c0.z = static_cast<uint32_t>(q >> 32);
                         cw[lane] = c0;
                     }
                     if (v1) {
-                        const uint64_t q = quantize_fast(c1.x, shift);
+                        const uint64_t q = quantize_energy(c1.x, shift);
                         c1.y = static_cast<uint32_t>(q);
                         c1.z = static_cast<uint32_t>(q >> 32);
                         cw[lane + 32] = c1;
@@ -346,12 +323,12 @@ select_mask_kernel(const __grid_constant__ SelectParams p) {
                     }
                     const uint32_t ustar =
                         warp_max_u32(max((v0 && G0 >= T) ? c0.x : 0u, (v1 && G1 >= T) ? c1.x : 0u));
-                    const uint64_t v = quantize_fast(ustar, shift);       // > 0 (see above)
+                    const uint64_t v = quantize_energy(ustar, shift);       // > 0 (see above)
                     // 4. no block outside bin k* may tie with v
                     const uint32_t top = btop - kstar;
                     const uint32_t lo_p = top << 22, hi_p = (top + 1) << 22;
-                    const bool straddle = (lo_p > 0 && quantize_fast(lo_p - 1, shift) == v) ||
-                                          quantize_fast(hi_p, shift) == v;
+                    const bool straddle = (lo_p > 0 && quantize_energy(lo_p - 1, shift) == v) ||
+                                          quantize_energy(hi_p, shift) == v;
                     if (!straddle && v != 0) {
                         const uint64_t q0 = (static_cast<uint64_t>(c0.z) << 32) | c0.y;
                         const uint64_t q1 = (static_cast<uint64_t>(c1.z) << 32) | c1.y;
@@ -393,7 +370,7 @@ select_mask_kernel(const __grid_constant__ SelectParams p) {
                         for (int x = static_cast<int>(lane); x < 32 * MPL; x += 32) {
                             const uint32_t bx = rb[x];
                             if (bx >= u) {
-                                const uint64_t q = quantize_fast(bx, shift);
+                                const uint64_t q = quantize_energy(bx, shift);
                                 sl += static_cast<uint32_t>(q) & lomask;
                                 sh += static_cast<uint32_t>(q >> cs);
                             }
@@ -406,14 +383,14 @@ select_mask_kernel(const __grid_constant__ SelectParams p) {
                         if (G_all(mid) >= T) ul = mid;
                         else uh = mid;
                     }
-                    const uint64_t v = quantize_fast(ul, shift);
+                    const uint64_t v = quantize_energy(ul, shift);
                     // free blocks above v are kept; ties at v in index order (this lane's
                     // blocks are j0 .. j0 + MPL - 1)
                     uint32_t gl = 0, gh = 0, ce = 0, eqbits = 0;
 #pragma unroll 1
                     for (int m = 0; m < MPL; ++m) {
                         const uint32_t bx = rb[j0 + m];              // forced and padding: 0
-                        const uint64_t q = bx ? quantize_fast(bx, shift) : 0ull;
+                        const uint64_t q = bx ? quantize_energy(bx, shift) : 0ull;
                         if (q > v) {
                             kbits |= 1u << m;
                             gl += static_cast<uint32_t>(q) & lomask;
