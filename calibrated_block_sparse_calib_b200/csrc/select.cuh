@@ -2,6 +2,7 @@
 // schedule and anchor-row list.  HBM-light kernels: one warp per (head, query block) row.
 #pragma once
 #include <cstdint>
+#include <type_traits>
 #include "ptx.cuh"
 
 namespace calib {
@@ -81,15 +82,19 @@ __device__ __forceinline__ uint64_t warp_exclusive_scan_u64(uint64_t v) {
 // This is the same integer as rounding the significand shifted by E' - 150 + shift bits
 // (E' = max(E, 1)) with round-half-even on the bits shifted out; a CPU check compared the
 // two on every exponent and on exact halves.
+template <bool SUBNORMAL = true>
 __device__ __forceinline__ uint64_t quantize_energy(uint32_t x, int shift) {
     const uint32_t E = x >> 23;
     const uint32_t hi = ((E + 896u + static_cast<uint32_t>(shift)) << 20) | ((x & 0x7FFFFFu) >> 3);
-    const double dn = __hiloint2double(static_cast<int>(hi), static_cast<int>(x << 29));
-    // a subnormal x is its significand times 2^-149: an exact integer conversion and an exact
-    // scaling by a power of two (built from its exponent field)
-    const double ds = __dmul_rn(__uint2double_rn(x & 0x7FFFFFu),
-                                __hiloint2double(static_cast<int>((874u + static_cast<uint32_t>(shift)) << 20), 0));
-    const double r = __dadd_rn(E ? dn : ds, 4503599627370496.0);  // + 2^52
+    double d = __hiloint2double(static_cast<int>(hi), static_cast<int>(x << 29));
+    if constexpr (SUBNORMAL) {
+        // a subnormal x is its significand times 2^-149: an exact integer conversion and an
+        // exact scaling by a power of two (built from its exponent field)
+        const double ds = __dmul_rn(__uint2double_rn(x & 0x7FFFFFu),
+                                    __hiloint2double(static_cast<int>((874u + static_cast<uint32_t>(shift)) << 20), 0));
+        d = E ? d : ds;
+    }
+    const double r = __dadd_rn(d, 4503599627370496.0);            // + 2^52
     return static_cast<uint64_t>(__double_as_longlong(r)) & 0xFFFFFFFFFFFFFull;
 }
 
@@ -230,27 +235,31 @@ select_mask_kernel(const __grid_constant__ SelectParams p) {
             bmax = warp_max_u32(bmax);
             const uint32_t btop = bmax >> 22;                 // bin 0: the top half level
             // 1. histogram of the free blocks' q by half level below the top
+            // Blocks with q > 0 lie within 107 bins of the top; a block further down has q = 0,
+            // and clamping its bin to the last one adds nothing there.  It can become a
+            // candidate only if the answer lies in that last bin, where its q = 0 keeps it out
+            // of the kept set (v > 0).
             uint32_t dm[MPL];                                 // bin of each block, 0xFF: none
 #pragma unroll
             for (int m = 0; m < MPL; ++m) dm[m] = 0xFFu;
-            bool far = false;
             const uint32_t hlo_a = smem_u32(hlo), hhi_a = smem_u32(hhi);
+            bool sub = false;                                 // any subnormal free energy?
 #pragma unroll
-            for (int m = 0; m < MPL; ++m) {
-                if (b[m] != 0u) {
-                    const uint64_t q = quantize_energy(b[m], shift);
-                    if (q != 0) {
-                        const uint32_t d = btop - (b[m] >> 22);
-                        if (d < static_cast<uint32_t>(NB)) {
-                            red_shared_add(hlo_a + 4 * d, static_cast<uint32_t>(q) & lomask);
-                            red_shared_add(hhi_a + 4 * d, static_cast<uint32_t>(q >> cs));
-                            dm[m] = d;
-                        } else {
-                            far = true;                      // cannot happen (q > 0 implies d <= 107)
-                        }
+            for (int m = 0; m < MPL; ++m) sub |= b[m] != 0u && (b[m] >> 23) == 0u;
+            auto add_bins = [&](auto subnormal) {
+#pragma unroll
+                for (int m = 0; m < MPL; ++m) {
+                    if (b[m] != 0u) {
+                        const uint64_t q = quantize_energy<decltype(subnormal)::value>(b[m], shift);
+                        const uint32_t d = min(btop - (b[m] >> 22), static_cast<uint32_t>(NB - 1));
+                        red_shared_add(hlo_a + 4 * d, static_cast<uint32_t>(q) & lomask);
+                        red_shared_add(hhi_a + 4 * d, static_cast<uint32_t>(q >> cs));
+                        dm[m] = d;
                     }
                 }
-            }
+            };
+            if (__any_sync(0xffffffffu, sub)) add_bins(std::true_type{});
+            else add_bins(std::false_type{});
             __syncwarp();
             // 2. scan of the bins (lane l: bins 4l .. 4l+3), clearing them for the next row
             const uint4 lo4 = reinterpret_cast<const uint4*>(hlo)[lane];
@@ -266,7 +275,6 @@ select_mask_kernel(const __grid_constant__ SelectParams p) {
             const uint64_t Q = F + Qf;
             uint64_t T = __double2ull_rz(ceil(__dmul_rn(p.tau[bi], __ull2double_rn(Q))));
             if (T < 1) T = 1;
-            far = __any_sync(0xffffffffu, far);
             if (F < T) {
                 // first bin whose cumulative sum reaches T
                 const uint64_t C = F + base;
@@ -285,7 +293,7 @@ select_mask_kernel(const __grid_constant__ SelectParams p) {
                 const uint32_t cl = __popc(cmask);
                 const uint32_t nc = warp_sum_u32(cl);
                 bool done = false;
-                if (!far && nc <= static_cast<uint32_t>(kSelCompact)) {
+                if (nc <= static_cast<uint32_t>(kSelCompact)) {
                     const uint32_t pos0 = warp_exclusive_scan(cl);
                     uint4* cw = cand[wib];
                     // each block's slot is fixed by the blocks before it (so the slots are in
@@ -345,11 +353,14 @@ select_mask_kernel(const __grid_constant__ SelectParams p) {
                         if (gt0 || (eq0 && r0 < need)) red_shared_or(km_a + 4 * (c0.w >> 5), 1u << (c0.w & 31));
                         if (gt1 || (eq1 && r1 < need)) red_shared_or(km_a + 4 * (c1.w >> 5), 1u << (c1.w & 31));
                         __syncwarp();
+                        // this lane's blocks j0 .. j0 + MPL - 1 lie in at most two mask words
+                        const uint32_t w0 = kmask[wib][j0 >> 5];
+                        const uint32_t w1 = kmask[wib][min(j0 + MPL - 1, 32 * 32 - 1) >> 5];
+                        const uint64_t wins = ((static_cast<uint64_t>(w1) << 32) | w0) >> (j0 & 31);
 #pragma unroll
                         for (int m = 0; m < MPL; ++m) {
                             const uint32_t d = dm[m];
-                            const int j = j0 + m;
-                            const bool k = d < kstar || (d == kstar && ((kmask[wib][j >> 5] >> (j & 31)) & 1u));
+                            const bool k = d < kstar || (d == kstar && ((wins >> m) & 1ull));
                             kbits |= (k ? 1u : 0u) << m;
                         }
                         done = true;
