@@ -217,8 +217,9 @@ select_mask_kernel(const __grid_constant__ SelectParams p) {
         } else {
             const int shift = 52 - float_exponent_p(xmax) - c;
             // forced blocks: their q counts toward F; they are not free (pattern 0)
-            uint32_t fl = 0, fh = 0, bmax = 0;
+            uint64_t F = 0;
             if (__any_sync(0xffffffffu, fbits != 0u)) {
+                uint32_t fl = 0, fh = 0;
 #pragma unroll
                 for (int m = 0; m < MPL; ++m) {
                     if ((fbits >> m) & 1u) {
@@ -228,10 +229,11 @@ select_mask_kernel(const __grid_constant__ SelectParams p) {
                         b[m] = 0u;
                     }
                 }
+                F = join(warp_sum_u32(fh), warp_sum_u32(fl));
             }
+            uint32_t bmax = 0;
 #pragma unroll
             for (int m = 0; m < MPL; ++m) bmax = b[m] > bmax ? b[m] : bmax;
-            const uint64_t F = join(warp_sum_u32(fh), warp_sum_u32(fl));
             bmax = warp_max_u32(bmax);
             const uint32_t btop = bmax >> 22;                 // bin 0: the top half level
             // 1. histogram of the free blocks' q by half level below the top
@@ -343,15 +345,15 @@ select_mask_kernel(const __grid_constant__ SelectParams p) {
                         const bool gt0 = v0 && q0 > v, gt1 = v1 && q1 > v;
                         const bool eq0 = v0 && q0 == v, eq1 = v1 && q1 == v;
                         const uint64_t R = T - A - warp_sum_u64((gt0 ? q0 : 0ull) + (gt1 ? q1 : 0ull));   // > 0
-                        // exact ceil(R / v): a float estimate, then integer steps (R <= nk * v)
-                        uint64_t need = static_cast<uint64_t>(__fdividef(__ull2float_rn(R), __ull2float_rn(v)));
-                        while (need * v < R) ++need;
-                        while (need > 0 && (need - 1) * v >= R) --need;
+                        // ties in index order: the tie of rank r is kept iff the r ties before it
+                        // leave the sum short of T, r * v < R (the first ceil(R / v) of them)
                         const uint32_t e0 = __ballot_sync(0xffffffffu, eq0), e1 = __ballot_sync(0xffffffffu, eq1);
                         const uint32_t r0 = __popc(e0 & lanemask_lt()), r1 = __popc(e0) + __popc(e1 & lanemask_lt());
                         const uint32_t km_a = smem_u32(kmask[wib]);
-                        if (gt0 || (eq0 && r0 < need)) red_shared_or(km_a + 4 * (c0.w >> 5), 1u << (c0.w & 31));
-                        if (gt1 || (eq1 && r1 < need)) red_shared_or(km_a + 4 * (c1.w >> 5), 1u << (c1.w & 31));
+                        if (gt0 || (eq0 && static_cast<uint64_t>(r0) * v < R))
+                            red_shared_or(km_a + 4 * (c0.w >> 5), 1u << (c0.w & 31));
+                        if (gt1 || (eq1 && static_cast<uint64_t>(r1) * v < R))
+                            red_shared_or(km_a + 4 * (c1.w >> 5), 1u << (c1.w & 31));
                         __syncwarp();
                         // this lane's blocks j0 .. j0 + MPL - 1 lie in at most two mask words
                         const uint32_t w0 = kmask[wib][j0 >> 5];
