@@ -73,21 +73,23 @@ __device__ __forceinline__ uint64_t warp_exclusive_scan_u64(uint64_t v) {
     return x - v;
 }
 
-// q = rint(e * 2^shift), ties to even, for e >= 0 given by its binary32 bits x, computed
-// on the FP64 pipe.  For a normal x (exponent field E >= 1) the binary64 with exponent
-// E + 896 + shift and x's significand is exactly e * 2^shift (no overflow or underflow for
-// shift in [-86, 200]).  A subnormal x is its significand times 2^-149: an exact integer
-// conversion scaled by an exact power of two.  Adding 2^52 then rounds the product to an
-// integer, half to even (e * 2^shift < 2^52 here), and q is the low 52 bits of the sum.
-// This is the same integer as rounding the significand shifted by E' - 150 + shift bits
-// (E' = max(E, 1)) with round-half-even on the bits shifted out; a CPU check compared the
-// two on every exponent and on exact halves.
+// q = rint(e * 2^shift), ties to even, for e >= 0 given by its binary32 bits x < 2^31,
+// computed on the FP64 pipe.  For a normal x (exponent field E >= 1) the binary64 with
+// exponent E + 896 + shift and x's significand is exactly e * 2^shift (no overflow or
+// underflow for shift in [-86, 200]).  x >> 3 holds E in bits 20..27 above the top 20 bits
+// of the significand, so one integer add of (896 + shift) << 20 gives that binary64's high
+// word.  A subnormal x is its significand times 2^-149: an exact integer conversion scaled
+// by an exact power of two.  Adding 2^52 then rounds the product to an integer, half to
+// even (e * 2^shift < 2^52 here), and q is the low 52 bits of the sum.  This is the same
+// integer as rounding the significand shifted by E' - 150 + shift bits (E' = max(E, 1))
+// with round-half-even on the bits shifted out; a CPU check compared the two on every
+// exponent and on exact halves.
 template <bool SUBNORMAL = true>
 __device__ __forceinline__ uint64_t quantize_energy(uint32_t x, int shift) {
-    const uint32_t E = x >> 23;
-    const uint32_t hi = ((E + 896u + static_cast<uint32_t>(shift)) << 20) | ((x & 0x7FFFFFu) >> 3);
+    const uint32_t hi = (x >> 3) + ((896u + static_cast<uint32_t>(shift)) << 20);
     double d = __hiloint2double(static_cast<int>(hi), static_cast<int>(x << 29));
     if constexpr (SUBNORMAL) {
+        const uint32_t E = x >> 23;
         // a subnormal x is its significand times 2^-149: an exact integer conversion and an
         // exact scaling by a power of two (built from its exponent field)
         const double ds = __dmul_rn(__uint2double_rn(x & 0x7FFFFFu),
@@ -197,17 +199,24 @@ select_mask_kernel(const __grid_constant__ SelectParams p) {
 #pragma unroll
             for (int m = 0; m < MPL; ++m) b[m] = j0 + m < nk ? __float_as_uint(E[j0 + m]) : 0u;
         }
-        // negative, NaN or infinite energies count as 0 (and are reported); -0 becomes +0
-        bool bad = false;
+        // Patterns below +inf's (0x7F800000) are +0 and the finite positive energies.  Only
+        // a warp holding a larger pattern sanitises: negative, NaN or infinite energies
+        // count as 0 (and are reported); -0 becomes +0.
         uint32_t xmax = 0;
 #pragma unroll
-        for (int m = 0; m < MPL; ++m) {
-            const float x = __uint_as_float(b[m]);
-            if (!(x >= 0.f) || x == INFINITY) bad = true;
-            if (!(x > 0.f) || x == INFINITY) b[m] = 0u;
-            xmax = b[m] > xmax ? b[m] : xmax;
+        for (int m = 0; m < MPL; ++m) xmax = b[m] > xmax ? b[m] : xmax;
+        if (__any_sync(0xffffffffu, xmax >= 0x7F800000u)) {
+            bool bad = false;
+            xmax = 0;
+#pragma unroll
+            for (int m = 0; m < MPL; ++m) {
+                const float x = __uint_as_float(b[m]);
+                if (!(x >= 0.f) || x == INFINITY) bad = true;
+                if (!(x > 0.f) || x == INFINITY) b[m] = 0u;
+                xmax = b[m] > xmax ? b[m] : xmax;
+            }
+            if (__any_sync(0xffffffffu, bad) && lane == 0) raise_status(STATUS_BAD_ENERGY);
         }
-        if (__any_sync(0xffffffffu, bad) && lane == 0) raise_status(STATUS_BAD_ENERGY);
         xmax = warp_max_u32(xmax);
 
         uint32_t kbits = fbits;
@@ -218,6 +227,7 @@ select_mask_kernel(const __grid_constant__ SelectParams p) {
             const int shift = 52 - float_exponent_p(xmax) - c;
             // forced blocks: their q counts toward F; they are not free (pattern 0)
             uint64_t F = 0;
+            uint32_t bmax = xmax;                             // largest free pattern
             if (__any_sync(0xffffffffu, fbits != 0u)) {
                 uint32_t fl = 0, fh = 0;
 #pragma unroll
@@ -230,24 +240,21 @@ select_mask_kernel(const __grid_constant__ SelectParams p) {
                     }
                 }
                 F = join(warp_sum_u32(fh), warp_sum_u32(fl));
-            }
-            uint32_t bmax = 0;
+                bmax = 0;
 #pragma unroll
-            for (int m = 0; m < MPL; ++m) bmax = b[m] > bmax ? b[m] : bmax;
-            bmax = warp_max_u32(bmax);
+                for (int m = 0; m < MPL; ++m) bmax = b[m] > bmax ? b[m] : bmax;
+                bmax = warp_max_u32(bmax);
+            }
             const uint32_t btop = bmax >> 22;                 // bin 0: the top half level
             // 1. histogram of the free blocks' q by half level below the top
             // Blocks with q > 0 lie within 107 bins of the top; a block further down has q = 0,
             // and clamping its bin to the last one adds nothing there.  It can become a
             // candidate only if the answer lies in that last bin, where its q = 0 keeps it out
             // of the kept set (v > 0).
-            uint32_t dm[MPL];                                 // bin of each block, 0xFF: none
-#pragma unroll
-            for (int m = 0; m < MPL; ++m) dm[m] = 0xFFu;
             const uint32_t hlo_a = smem_u32(hlo), hhi_a = smem_u32(hhi);
             bool sub = false;                                 // any subnormal free energy?
 #pragma unroll
-            for (int m = 0; m < MPL; ++m) sub |= b[m] != 0u && (b[m] >> 23) == 0u;
+            for (int m = 0; m < MPL; ++m) sub |= b[m] - 1u < 0x7FFFFFu;   // 1 <= b < 2^23
             auto add_bins = [&](auto subnormal) {
 #pragma unroll
                 for (int m = 0; m < MPL; ++m) {
@@ -256,7 +263,6 @@ select_mask_kernel(const __grid_constant__ SelectParams p) {
                         const uint32_t d = min(btop - (b[m] >> 22), static_cast<uint32_t>(NB - 1));
                         red_shared_add(hlo_a + 4 * d, static_cast<uint32_t>(q) & lomask);
                         red_shared_add(hhi_a + 4 * d, static_cast<uint32_t>(q >> cs));
-                        dm[m] = d;
                     }
                 }
             };
@@ -287,11 +293,18 @@ select_mask_kernel(const __grid_constant__ SelectParams p) {
                 const uint64_t Aown = C + (kl == 0 ? 0 : (kl == 1 ? p0 : (kl == 2 ? p1 : p2)));
                 const uint64_t A = __shfl_sync(0xffffffffu, Aown, L);        // G(top of bin k*)
                 const uint32_t kstar = static_cast<uint32_t>(4 * L + kls);
+                // bin k* holds the free patterns in [in_lo, hi_p): the last bin also every
+                // pattern below its top, and no bin holds pattern 0 (forced, zero, padding)
+                const uint32_t top = btop - kstar;
+                const uint32_t lo_p = top << 22, hi_p = (top + 1) << 22;
+                const uint32_t in_lo = kstar == static_cast<uint32_t>(NB - 1) ? 1u : (lo_p > 0u ? lo_p : 1u);
                 // 3. the blocks of bin k*, in index order
-                uint32_t cmask = 0;                          // this lane's blocks in bin k*
+                uint32_t cmask = 0, above = 0;               // this lane's blocks in / above bin k*
 #pragma unroll
-                for (int m = 0; m < MPL; ++m)
-                    cmask |= (dm[m] == kstar ? 1u : 0u) << m;
+                for (int m = 0; m < MPL; ++m) {
+                    cmask |= (b[m] >= in_lo && b[m] < hi_p ? 1u : 0u) << m;
+                    above |= (b[m] >= hi_p ? 1u : 0u) << m;
+                }
                 const uint32_t cl = __popc(cmask);
                 const uint32_t nc = warp_sum_u32(cl);
                 bool done = false;
@@ -335,8 +348,6 @@ select_mask_kernel(const __grid_constant__ SelectParams p) {
                         warp_max_u32(max((v0 && G0 >= T) ? c0.x : 0u, (v1 && G1 >= T) ? c1.x : 0u));
                     const uint64_t v = quantize_energy(ustar, shift);       // > 0 (see above)
                     // 4. no block outside bin k* may tie with v
-                    const uint32_t top = btop - kstar;
-                    const uint32_t lo_p = top << 22, hi_p = (top + 1) << 22;
                     const bool straddle = (lo_p > 0 && quantize_energy(lo_p - 1, shift) == v) ||
                                           quantize_energy(hi_p, shift) == v;
                     if (!straddle && v != 0) {
@@ -355,16 +366,13 @@ select_mask_kernel(const __grid_constant__ SelectParams p) {
                         if (gt1 || (eq1 && static_cast<uint64_t>(r1) * v < R))
                             red_shared_or(km_a + 4 * (c1.w >> 5), 1u << (c1.w & 31));
                         __syncwarp();
-                        // this lane's blocks j0 .. j0 + MPL - 1 lie in at most two mask words
+                        // this lane's blocks j0 .. j0 + MPL - 1 lie in at most two mask words,
+                        // where only blocks of bin k* have bits
                         const uint32_t w0 = kmask[wib][j0 >> 5];
                         const uint32_t w1 = kmask[wib][min(j0 + MPL - 1, 32 * 32 - 1) >> 5];
                         const uint64_t wins = ((static_cast<uint64_t>(w1) << 32) | w0) >> (j0 & 31);
-#pragma unroll
-                        for (int m = 0; m < MPL; ++m) {
-                            const uint32_t d = dm[m];
-                            const bool k = d < kstar || (d == kstar && ((wins >> m) & 1ull));
-                            kbits |= (k ? 1u : 0u) << m;
-                        }
+                        const uint32_t lanebits = MPL >= 32 ? 0xFFFFFFFFu : ((1u << MPL) - 1u);
+                        kbits |= above | (static_cast<uint32_t>(wins) & lanebits);
                         done = true;
                     }
                     __syncwarp();                                 // candidates read before reuse
@@ -439,9 +447,10 @@ select_mask_kernel(const __grid_constant__ SelectParams p) {
 #pragma unroll
                     for (int v = 0; v < MPL / 4; ++v) {
                         if (j0 + 4 * v < nk) {
+                            // bit i of x times 1 + 2^7 + 2^14 + 2^21 lands at bit 8i (the
+                            // sixteen products sit at distinct bits: no carries)
                             const uint32_t x = (kbits >> (4 * v)) & 0xFu;
-                            reinterpret_cast<uint32_t*>(M + j0)[v] =
-                                (x & 1u) | ((x & 2u) << 7) | ((x & 4u) << 14) | ((x & 8u) << 21);
+                            reinterpret_cast<uint32_t*>(M + j0)[v] = (x * 0x00204081u) & 0x01010101u;
                         }
                     }
                 }
