@@ -55,12 +55,6 @@ __device__ __forceinline__ int float_exponent_p(uint32_t bits) {
     return msb - 148;
 }
 
-// 64-bit sum over the lanes of a warp (butterfly of 32-bit shuffles).
-__device__ __forceinline__ uint64_t warp_sum_u64(uint64_t v) {
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
-    return v;
-}
 // Exclusive prefix sum of 64-bit values over the lanes of a warp.
 __device__ __forceinline__ uint64_t warp_exclusive_scan_u64(uint64_t v) {
     const uint32_t lane = lane_id();
@@ -101,8 +95,11 @@ __device__ __forceinline__ uint64_t quantize_energy(uint32_t x, int shift) {
 }
 
 // Shared-memory reductions by shared-space address (no generic-address check).
-__device__ __forceinline__ void red_shared_add(uint32_t addr, uint32_t v) {
-    asm volatile("red.shared.add.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+// Adds lo at addr and hi at addr + OFF (one base register, an immediate offset).
+template <int OFF>
+__device__ __forceinline__ void red_shared_add_pair(uint32_t addr, uint32_t lo, uint32_t hi) {
+    asm volatile("red.shared.add.u32 [%0], %1;\n\tred.shared.add.u32 [%0+%3], %2;"
+                 ::"r"(addr), "r"(lo), "r"(hi), "n"(OFF) : "memory");
 }
 __device__ __forceinline__ void red_shared_or(uint32_t addr, uint32_t v) {
     asm volatile("red.shared.or.b32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
@@ -141,8 +138,7 @@ __global__ void __launch_bounds__(kSelWarps * 32, MPL <= 8 ? 8 : (MPL <= 16 ? 6 
 select_mask_kernel(const __grid_constant__ SelectParams p) {
     static_assert(MPL >= 1 && MPL <= kSelMaxPerLane, "per-lane count");
     constexpr int NB = kSelBins;
-    __shared__ __align__(16) uint32_t hist_lo[kSelWarps][NB];
-    __shared__ __align__(16) uint32_t hist_hi[kSelWarps][NB];
+    __shared__ __align__(16) uint32_t hist[kSelWarps][2 * NB];     // low parts, then high parts
     __shared__ __align__(16) uint4 cand[kSelWarps][kSelCompact];   // (b, q low, q high, j)
     __shared__ uint32_t kmask[kSelWarps][32];                      // kept candidates, by j
     __shared__ uint32_t rowb[kSelWarps][32 * MPL];                 // the row's patterns (fallback)
@@ -163,8 +159,8 @@ select_mask_kernel(const __grid_constant__ SelectParams p) {
     auto join = [&](uint32_t hi_sum, uint32_t lo_sum) -> uint64_t {
         return (static_cast<uint64_t>(hi_sum) << cs) + lo_sum;
     };
-    uint32_t* hlo = hist_lo[wib];
-    uint32_t* hhi = hist_hi[wib];
+    uint32_t* hlo = hist[wib];
+    uint32_t* hhi = hist[wib] + NB;
     reinterpret_cast<uint4*>(hlo)[lane] = make_uint4(0, 0, 0, 0);  // bins 4*lane .. 4*lane+3
     reinterpret_cast<uint4*>(hhi)[lane] = make_uint4(0, 0, 0, 0);
     __syncwarp();
@@ -251,18 +247,22 @@ select_mask_kernel(const __grid_constant__ SelectParams p) {
             // and clamping its bin to the last one adds nothing there.  It can become a
             // candidate only if the answer lies in that last bin, where its q = 0 keeps it out
             // of the kept set (v > 0).
-            const uint32_t hlo_a = smem_u32(hlo), hhi_a = smem_u32(hhi);
-            bool sub = false;                                 // any subnormal free energy?
+            // bin d = min(btop - (b >> 22), NB - 1) of a free block (b <= bmax) sits at
+            // a_top - 4 * (b >> 22), clamped to the last bin's address
+            const uint32_t a_top = smem_u32(hlo) + 4u * btop, a_last = smem_u32(hlo) + 4u * (NB - 1);
+            uint32_t bm1 = 0xFFFFFFFFu;                       // smallest free pattern minus 1
 #pragma unroll
-            for (int m = 0; m < MPL; ++m) sub |= b[m] - 1u < 0x7FFFFFu;   // 1 <= b < 2^23
+            for (int m = 0; m < MPL; ++m) bm1 = min(bm1, b[m] - 1u);
+            const bool sub = bm1 < 0x7FFFFFu;                 // a subnormal free energy: 1 <= b < 2^23
             auto add_bins = [&](auto subnormal) {
 #pragma unroll
                 for (int m = 0; m < MPL; ++m) {
                     if (b[m] != 0u) {
                         const uint64_t q = quantize_energy<decltype(subnormal)::value>(b[m], shift);
-                        const uint32_t d = min(btop - (b[m] >> 22), static_cast<uint32_t>(NB - 1));
-                        red_shared_add(hlo_a + 4 * d, static_cast<uint32_t>(q) & lomask);
-                        red_shared_add(hhi_a + 4 * d, static_cast<uint32_t>(q >> cs));
+                        const uint32_t a = min(a_top - 4u * (b[m] >> 22), a_last);
+                        red_shared_add_pair<4 * NB>(a, static_cast<uint32_t>(q) & lomask,
+                                                    __funnelshift_rc(static_cast<uint32_t>(q),
+                                                                     static_cast<uint32_t>(q >> 32), cs));
                     }
                 }
             };
@@ -286,7 +286,8 @@ select_mask_kernel(const __grid_constant__ SelectParams p) {
             if (F < T) {
                 // first bin whose cumulative sum reaches T
                 const uint64_t C = F + base;
-                const int kl = C + p0 >= T ? 0 : (C + p1 >= T ? 1 : (C + p2 >= T ? 2 : (C + p3 >= T ? 3 : 4)));
+                const uint64_t gap = C >= T ? 0ull : T - C;   // C + p_k >= T  <=>  p_k >= gap
+                const int kl = p0 >= gap ? 0 : (p1 >= gap ? 1 : (p2 >= gap ? 2 : (p3 >= gap ? 3 : 4)));
                 const uint32_t has = __ballot_sync(0xffffffffu, kl < 4);   // non-empty: the total reaches T
                 const int L = __ffs(has) - 1;
                 const int kls = __shfl_sync(0xffffffffu, kl, L);
@@ -313,11 +314,10 @@ select_mask_kernel(const __grid_constant__ SelectParams p) {
                     uint4* cw = cand[wib];
                     // each block's slot is fixed by the blocks before it (so the slots are in
                     // index order); its q is filled in by the lane that reads the slot
+                    uint32_t pos = pos0;
 #pragma unroll
                     for (int m = 0; m < MPL; ++m)
-                        if ((cmask >> m) & 1u)
-                            cw[pos0 + __popc(cmask & ((1u << m) - 1u))] =
-                                make_uint4(b[m], 0u, 0u, static_cast<uint32_t>(j0 + m));
+                        if ((cmask >> m) & 1u) cw[pos++] = make_uint4(b[m], 0u, 0u, static_cast<uint32_t>(j0 + m));
                     kmask[wib][lane] = 0u;
                     __syncwarp();
                     const bool v0 = lane < nc, v1 = lane + 32 < nc;
@@ -355,7 +355,12 @@ select_mask_kernel(const __grid_constant__ SelectParams p) {
                         const uint64_t q1 = (static_cast<uint64_t>(c1.z) << 32) | c1.y;
                         const bool gt0 = v0 && q0 > v, gt1 = v1 && q1 > v;
                         const bool eq0 = v0 && q0 == v, eq1 = v1 && q1 == v;
-                        const uint64_t R = T - A - warp_sum_u64((gt0 ? q0 : 0ull) + (gt1 ? q1 : 0ull));   // > 0
+                        // the sum of q over the kept candidates, in the histogram's two 32-bit parts
+                        const uint32_t gl = (gt0 ? static_cast<uint32_t>(q0) & lomask : 0u) +
+                                            (gt1 ? static_cast<uint32_t>(q1) & lomask : 0u);
+                        const uint32_t gh = (gt0 ? __funnelshift_rc(c0.y, c0.z, cs) : 0u) +
+                                            (gt1 ? __funnelshift_rc(c1.y, c1.z, cs) : 0u);
+                        const uint64_t R = T - A - join(warp_sum_u32(gh), warp_sum_u32(gl));   // > 0
                         // ties in index order: the tie of rank r is kept iff the r ties before it
                         // leave the sum short of T, r * v < R (the first ceil(R / v) of them)
                         const uint32_t e0 = __ballot_sync(0xffffffffu, eq0), e1 = __ballot_sync(0xffffffffu, eq1);
