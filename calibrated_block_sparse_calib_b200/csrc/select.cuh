@@ -94,6 +94,11 @@ __device__ __forceinline__ uint64_t quantize_energy(uint32_t x, int shift) {
     return static_cast<uint64_t>(__double_as_longlong(r)) & 0xFFFFFFFFFFFFFull;
 }
 
+// Position of word w of a row staged in shared memory: with PAD, 4 words of padding after
+// every 32, which keeps 4-word groups aligned and spreads the lanes' runs over the banks.
+template <bool PAD>
+__device__ __forceinline__ int staged_word(int w) { return PAD ? w + 4 * (w >> 5) : w; }
+
 // Shared-memory reductions by shared-space address (no generic-address check).
 // Adds lo at addr and hi at addr + OFF (one base register, an immediate offset).
 template <int OFF>
@@ -141,7 +146,11 @@ select_mask_kernel(const __grid_constant__ SelectParams p) {
     __shared__ __align__(16) uint32_t hist[kSelWarps][2 * NB];     // low parts, then high parts
     __shared__ __align__(16) uint4 cand[kSelWarps][kSelCompact];   // (b, q low, q high, j)
     __shared__ uint32_t kmask[kSelWarps][32];                      // kept candidates, by j
-    __shared__ uint32_t rowb[kSelWarps][32 * MPL];                 // the row's patterns (fallback)
+    // A row of words, for rows that are not 16-byte aligned and for the fallback.  Staged
+    // rows place word w at w + 4 * (w / 32) when MPL % 8 == 0: the lanes' 16-byte accesses at
+    // a stride of MPL words then fall on distinct banks.
+    constexpr bool PAD = MPL % 8 == 0;
+    __shared__ __align__(16) uint32_t rowb[kSelWarps][(PAD ? 36 : 32) * MPL];
     const uint32_t wib = warp_id();
     const long long gw = static_cast<long long>(blockIdx.x) * kSelWarps + wib;
     if (gw >= static_cast<long long>(p.rows) * p.n_chunks) return;
@@ -189,9 +198,27 @@ select_mask_kernel(const __grid_constant__ SelectParams p) {
                     b[4 * v + 2] = __float_as_uint(x.z);
                     b[4 * v + 3] = __float_as_uint(x.w);
                 }
+            } else {
+                // rows not 16-byte aligned: coalesced 4-byte loads into the warp's row buffer,
+                // then each lane reads its run back with 16-byte shared loads
+                uint32_t* rb = rowb[wib];
+#pragma unroll
+                for (int k = 0; k < MPL; ++k) {
+                    const int j = 32 * k + static_cast<int>(lane);
+                    rb[staged_word<PAD>(j)] = j < nk ? __float_as_uint(E[j]) : 0u;
+                }
+                __syncwarp();
+#pragma unroll
+                for (int v = 0; v < MPL / 4; ++v) {
+                    const uint4 x = *reinterpret_cast<const uint4*>(rb + staged_word<PAD>(j0 + 4 * v));
+                    b[4 * v] = x.x;
+                    b[4 * v + 1] = x.y;
+                    b[4 * v + 2] = x.z;
+                    b[4 * v + 3] = x.w;
+                }
+                __syncwarp();                                // read before the buffer is reused
             }
-        }
-        if (!(MPL % 4 == 0) || !p.vec) {
+        } else {
 #pragma unroll
             for (int m = 0; m < MPL; ++m) b[m] = j0 + m < nk ? __float_as_uint(E[j0 + m]) : 0u;
         }
@@ -460,7 +487,28 @@ select_mask_kernel(const __grid_constant__ SelectParams p) {
                     }
                 }
             }
-            if (!(MPL % 4 == 0) || !p.vec) {
+            if constexpr (MPL % 4 == 0 && !PAD) {
+                if (!p.vec) {
+                    // rows not 4-byte aligned, at MPL = 4 or 20 (an odd number of words per
+                    // lane, so the lanes' word stores fall on distinct banks): the lane's mask
+                    // bytes go to the row buffer, then the warp stores the row with coalesced
+                    // byte stores.  At the other widths the lanes' own byte stores measured
+                    // faster.
+                    uint32_t* rb = rowb[wib];
+#pragma unroll
+                    for (int v = 0; v < MPL / 4; ++v)
+                        rb[(j0 >> 2) + v] = (((kbits >> (4 * v)) & 0xFu) * 0x00204081u) & 0x01010101u;
+                    __syncwarp();
+                    const uint8_t* rbb = reinterpret_cast<const uint8_t*>(rb);
+#pragma unroll
+                    for (int k = 0; k < MPL; ++k) {
+                        const int j = 32 * k + static_cast<int>(lane);
+                        if (j < nk) M[j] = rbb[j];
+                    }
+                    __syncwarp();                            // read before the buffer is reused
+                }
+            }
+            if (!(MPL % 4 == 0) || (PAD && !p.vec)) {
 #pragma unroll
                 for (int m = 0; m < MPL; ++m)
                     if (j0 + m < nk) M[j0 + m] = static_cast<uint8_t>((kbits >> m) & 1u);
