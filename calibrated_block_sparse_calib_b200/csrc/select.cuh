@@ -347,20 +347,24 @@ select_mask_kernel(const __grid_constant__ SelectParams p) {
                         if ((cmask >> m) & 1u) cw[pos++] = make_uint4(b[m], 0u, 0u, static_cast<uint32_t>(j0 + m));
                     kmask[wib][lane] = 0u;
                     __syncwarp();
-                    const bool v0 = lane < nc, v1 = lane + 32 < nc;
+                    const bool two = nc > 32;                    // second slot in use (warp-uniform)
+                    const bool v0 = lane < nc, v1 = two && lane + 32 < nc;
                     uint4 c0 = v0 ? cw[lane] : make_uint4(0, 0, 0, 0);
-                    uint4 c1 = v1 ? cw[lane + 32] : make_uint4(0, 0, 0, 0);
+                    uint4 c1 = make_uint4(0, 0, 0, 0);
                     if (v0) {
                         const uint64_t q = quantize_energy(c0.x, shift);
                         c0.y = static_cast<uint32_t>(q);
                         c0.z = static_cast<uint32_t>(q >> 32);
                         cw[lane] = c0;
                     }
-                    if (v1) {
-                        const uint64_t q = quantize_energy(c1.x, shift);
-                        c1.y = static_cast<uint32_t>(q);
-                        c1.z = static_cast<uint32_t>(q >> 32);
-                        cw[lane + 32] = c1;
+                    if (two) {
+                        if (v1) {
+                            c1 = cw[lane + 32];
+                            const uint64_t q = quantize_energy(c1.x, shift);
+                            c1.y = static_cast<uint32_t>(q);
+                            c1.z = static_cast<uint32_t>(q >> 32);
+                            cw[lane + 32] = c1;
+                        }
                     }
                     __syncwarp();
                     // G at each candidate's own pattern
@@ -369,34 +373,49 @@ select_mask_kernel(const __grid_constant__ SelectParams p) {
                         const uint4 e = cw[x];
                         const uint64_t qe = (static_cast<uint64_t>(e.z) << 32) | e.y;
                         if (e.x >= c0.x) G0 += qe;
-                        if (nc > 32 && e.x >= c1.x) G1 += qe;
+                        if (two && e.x >= c1.x) G1 += qe;
                     }
                     const uint32_t ustar =
                         warp_max_u32(max((v0 && G0 >= T) ? c0.x : 0u, (v1 && G1 >= T) ? c1.x : 0u));
                     const uint64_t v = quantize_energy(ustar, shift);       // > 0 (see above)
-                    // 4. no block outside bin k* may tie with v
-                    const bool straddle = (lo_p > 0 && quantize_energy(lo_p - 1, shift) == v) ||
-                                          quantize_energy(hi_p, shift) == v;
+                    // 4. no block outside bin k* may tie with v.  An energy of exponent field E
+                    // (E' = max(E, 1)) is an integer multiple of 2^(E' - 150), so where
+                    // E' - 150 + shift >= 0 at the pattern just below the bin, q is the exact
+                    // e * 2^shift from there up: distinct patterns give distinct q, and no block
+                    // outside the bin ties with v.  Otherwise the two patterns just outside the
+                    // bin are quantised.
+                    const uint32_t x_lo = lo_p > 0u ? lo_p - 1u : 0u;
+                    const bool exact = max(static_cast<int>(x_lo >> 23), 1) - 150 + shift >= 0;
+                    const bool straddle = !exact && ((lo_p > 0 && quantize_energy(lo_p - 1, shift) == v) ||
+                                                     quantize_energy(hi_p, shift) == v);
                     if (!straddle && v != 0) {
                         const uint64_t q0 = (static_cast<uint64_t>(c0.z) << 32) | c0.y;
-                        const uint64_t q1 = (static_cast<uint64_t>(c1.z) << 32) | c1.y;
-                        const bool gt0 = v0 && q0 > v, gt1 = v1 && q1 > v;
-                        const bool eq0 = v0 && q0 == v, eq1 = v1 && q1 == v;
+                        const bool gt0 = v0 && q0 > v, eq0 = v0 && q0 == v;
                         // the sum of q over the kept candidates, in the histogram's two 32-bit parts
-                        const uint32_t gl = (gt0 ? static_cast<uint32_t>(q0) & lomask : 0u) +
-                                            (gt1 ? static_cast<uint32_t>(q1) & lomask : 0u);
-                        const uint32_t gh = (gt0 ? __funnelshift_rc(c0.y, c0.z, cs) : 0u) +
-                                            (gt1 ? __funnelshift_rc(c1.y, c1.z, cs) : 0u);
+                        uint32_t gl = gt0 ? static_cast<uint32_t>(q0) & lomask : 0u;
+                        uint32_t gh = gt0 ? __funnelshift_rc(c0.y, c0.z, cs) : 0u;
+                        bool gt1 = false, eq1 = false;
+                        if (two) {
+                            const uint64_t q1 = (static_cast<uint64_t>(c1.z) << 32) | c1.y;
+                            gt1 = v1 && q1 > v;
+                            eq1 = v1 && q1 == v;
+                            gl += gt1 ? static_cast<uint32_t>(q1) & lomask : 0u;
+                            gh += gt1 ? __funnelshift_rc(c1.y, c1.z, cs) : 0u;
+                        }
                         const uint64_t R = T - A - join(warp_sum_u32(gh), warp_sum_u32(gl));   // > 0
                         // ties in index order: the tie of rank r is kept iff the r ties before it
                         // leave the sum short of T, r * v < R (the first ceil(R / v) of them)
-                        const uint32_t e0 = __ballot_sync(0xffffffffu, eq0), e1 = __ballot_sync(0xffffffffu, eq1);
-                        const uint32_t r0 = __popc(e0 & lanemask_lt()), r1 = __popc(e0) + __popc(e1 & lanemask_lt());
+                        const uint32_t e0 = __ballot_sync(0xffffffffu, eq0);
+                        const uint32_t r0 = __popc(e0 & lanemask_lt());
                         const uint32_t km_a = smem_u32(kmask[wib]);
                         if (gt0 || (eq0 && static_cast<uint64_t>(r0) * v < R))
                             red_shared_or(km_a + 4 * (c0.w >> 5), 1u << (c0.w & 31));
-                        if (gt1 || (eq1 && static_cast<uint64_t>(r1) * v < R))
-                            red_shared_or(km_a + 4 * (c1.w >> 5), 1u << (c1.w & 31));
+                        if (two) {
+                            const uint32_t e1 = __ballot_sync(0xffffffffu, eq1);
+                            const uint32_t r1 = __popc(e0) + __popc(e1 & lanemask_lt());
+                            if (gt1 || (eq1 && static_cast<uint64_t>(r1) * v < R))
+                                red_shared_or(km_a + 4 * (c1.w >> 5), 1u << (c1.w & 31));
+                        }
                         __syncwarp();
                         // this lane's blocks j0 .. j0 + MPL - 1 lie in at most two mask words,
                         // where only blocks of bin k* have bits

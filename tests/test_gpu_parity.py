@@ -187,6 +187,48 @@ def test_select_batched_bit_exact(nk):
     ops.device_check()
 
 
+def _coarse_rows(rng, nrows, nk):
+    """Rows of three blocks at 1.0 and tiny energies over six exponent levels, 2^-26 to 2^-35
+    of the maximum.  Their integers are coarser than the float spacing, so neighbouring
+    patterns share a q.  Half the tiny energies sit within 3 ulps of a half-level edge (a
+    pattern with the low 22 bits 0), half are spread over the level."""
+    out = np.zeros((nrows, nk), np.float32)
+    for r in range(nrows):
+        big = rng.choice(nk, size=3, replace=False)
+        e0 = int(rng.integers(26, 30))
+        lev = np.float32(2.0) ** -(e0 + rng.integers(0, 6, nk)).astype(np.float32)
+        near = lev * np.array([1.0, 1.5], np.float32)[rng.integers(0, 2, nk)]
+        ulp = rng.integers(-3, 4, nk).astype(np.int64)
+        near = (near.view(np.int32).astype(np.int64) + ulp).astype(np.int32).view(np.float32)
+        spread = (lev * (1.0 + rng.random(nk))).astype(np.float32)
+        x = np.where(rng.random(nk) < 0.5, near, spread).astype(np.float32)
+        x[big] = np.float32(1.0)
+        out[r] = x
+    return out
+
+
+@pytest.mark.parametrize("nk", [100, 256, 591])
+def test_select_coarse_quantisation_at_bin_edges(nk):
+    """Thresholds inside the tiny energies of _coarse_rows: tau puts T a tenth, half and nine
+    tenths of the way through their integer mass.  Ties between the threshold's bin and its
+    neighbours are possible there, so the kernel's check at the bin's edges decides both
+    ways across these rows (about a third take the exact bisection).  Each row is one batch
+    entry with its own tau; every mask equals the oracle's."""
+    rng = np.random.default_rng(4242 + nk)
+    e, taus = [], []
+    for r in _coarse_rows(rng, 40, nk):
+        qi, Q = oracle.quantize_row(r)
+        big = int(qi[r == np.float32(1.0)].sum())
+        for f in (0.1, 0.5, 0.9):
+            e.append(r)
+            taus.append(min(1.0, (big + f * (Q - big)) / Q))
+    e = np.stack(e)[:, None, None, :]
+    got = ops.select_mask_batched(torch.from_numpy(e).cuda(), taus).cpu().numpy()
+    for b, tau in enumerate(taus):
+        np.testing.assert_array_equal(got[b], oracle.select_mask(e[b], tau), err_msg=f"entry {b} tau {tau}")
+    ops.device_check()
+
+
 def test_select_batched_many_entries_split_over_warps():
     """Enough rows x entries that each row's entries are split into chunks handled by
     different warps (vote counts then combine atomically); counts only, no masks."""
