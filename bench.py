@@ -91,6 +91,20 @@ def kept_flops(mask: np.ndarray, N: int, D: int, B: int, repeat_heads=(), n_anch
     return 4.0 * D * total
 
 
+def workload_config(wl, mask_np, n_gpus: int, n_anchor) -> dict:
+    """The line's `config`, the same in both arms: the workload's shape, its kept fraction of
+    the dense FLOPs (repeat heads counted by their n_anchor anchor rows), and how the inputs
+    relate to L2."""
+    s = wl.shape
+    H, N, D, B = s.H, s.N, s.D, s.block
+    rep = tuple(h for h in range(H) if h in wl.repeat_heads)
+    density = kept_flops(mask_np, N, D, B, rep, n_anchor) / (4.0 * N * N * D * H)
+    qkvo_mb = 4 * H * N * D * 2 / 1e6
+    return {"workload": wl.name, "H": H, "N": N, "D": D, "block": B, "density": round(density, 4),
+            "repeat_heads": len(rep), "parallelism": f"replicas{n_gpus}",
+            "l2": f"inputs larger than L2 (Q/K/V/O {qkvo_mb:.0f} MB), no flush"}
+
+
 class ClockSampler:
     """nvidia-smi clock / throttle sampling during the timed region."""
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
@@ -308,7 +322,13 @@ def run_reference(args):
     from calibrated_block_sparse_calib_b200 import synth
     wl = synth.WORKLOADS[args.workload]
     q, k, v = synth.make_qkv(wl, heads=1)
-    mask = synth.make_head_masks(wl)[:1]
+    full_mask = synth.make_head_masks(wl, timestep=args.timestep)
+    mask = full_mask[:1]
+    n_anchor = None
+    if wl.repeat_heads:
+        import oracle
+        s = wl.shape
+        n_anchor = len(oracle.anchor_rows(s.F, s.Hl, s.Wl, s.n_text, wl.repeat_stride))
     per_step = []
     for _ in range(args.warmup):
         cpu_baseline(wl, q, k, v, mask, budget_s=0.5)
@@ -318,8 +338,7 @@ def run_reference(args):
     line = {"impl": "reference", "metric": METRIC, "value": val, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": wl.name, "H": wl.shape.H, "N": wl.shape.N, "D": wl.shape.D,
-                       "block": wl.shape.block},
+            "config": workload_config(wl, full_mask, args.gpus, n_anchor),
             "cpu_baseline": {"value": val, "unit": UNIT, "cores": per_step[0]["cores"], "kind": "oracle",
                              "sample": per_step[0]["sample"]},
             "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -692,10 +711,7 @@ def main():
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": wl.name, "H": H, "N": N, "D": D, "block": B, "density": round(density, 4),
-                   "repeat_heads": sum(rep), "parallelism": f"replicas{world}",
-                   "l2": f"inputs larger than L2 (Q/K/V/O {4 * q.numel() * q.element_size() / 1e6:.0f} MB), "
-                         "no flush"},
+        "config": workload_config(wl, mask_np, world, n_anchor),
         "dense_equiv_tflops": flops_dense * world / (ms * 1e-3) / 1e12,
         "frac_of_bf16_peak": value / world / peaks["bf16_tflops"],
         "roofline": {"bound": "tensor", "achieved": value / world, "peak": peaks["bf16_tflops"],
