@@ -15,15 +15,18 @@
 //               re-reads Q from shared memory for every key block, and at M=N=128 the
 //               operand reads, not the math, set its rate).  S rotates through three
 //               buffers; a buffer is handed back as soon as its tile is in registers.
-//   warps 2..9  arithmetic.  A query row (TMEM lane) is split between two warps, each
-//               owning half of every tile's columns.  Pass 1: each half keeps an exact
-//               running (max, sum) of 2^x over its columns; the halves are merged once, at
-//               the end of the pass, into the row's LSE (kept in a register: the LSE is
-//               never written to memory, so no scratch buffer is needed).  Pass 2: each
-//               thread sums 2^(x - lse2) over its columns; each warp reduces its 32 rows
-//               with shuffles, batched over four key blocks, into a shared-memory table of
-//               per-warp partials, and after the last key block the CTA adds the eight
-//               partials of every block in a fixed order and writes the row of energies.
+//   warps 2..9  arithmetic, in two groups of four warps (one per TMEM lane quadrant).
+//               Group g takes the tiles t with t % 2 == g, every column of each, so the two
+//               warps of a sub-partition work on different tiles and one's tensor-memory
+//               load and reduction overlap the other's exponentials.  Pass 1: each group
+//               keeps an exact running (max, sum) of 2^x over its tiles; the groups are
+//               merged once, at the end of the pass, into the row's LSE (kept in a register:
+//               the LSE is never written to memory, so no scratch buffer is needed).  Pass 2:
+//               each thread sums 2^(x - lse2) over a tile's columns; each warp reduces its 32
+//               rows with shuffles, batched over four of its group's key blocks, into a
+//               shared-memory table of per-warp partials, and after the last key block the
+//               CTA adds the four partials of every block (its group's warps) in a fixed
+//               order and writes the row of energies.
 // Tensor memory: S buffers at columns [0,128), [128,256), [256,384); Q at [384, 384+D/2).
 // [AdaSpa] §2 caches the LSE to reuse it in a later search; a supplied LSE skips pass 1.
 #pragma once
@@ -33,7 +36,7 @@
 
 namespace calib {
 
-constexpr int kEnergyGroups = 2;                          // column halves per row
+constexpr int kEnergyGroups = 2;                          // arithmetic groups (tile parity)
 constexpr int kEnergySoftmaxWarps = 4 * kEnergyGroups;    // 8
 constexpr int kEnergySoftmaxThreads = 32 * kEnergySoftmaxWarps;
 constexpr int kEnergyThreads = 64 + kEnergySoftmaxThreads;
@@ -74,7 +77,7 @@ __global__ void __launch_bounds__(kEnergyThreads, 1)
 block_energy_kernel(const __grid_constant__ CUtensorMap tm_k, const EnergyParams p) {
     using L = EnergySmem<D, BLK, KST>;
     constexpr int CH = L::CH;
-    constexpr int HC = BLK / kEnergyGroups;               // columns per thread and tile
+    constexpr int HC = BLK;                               // columns per thread and tile
     constexpr int SB = kEnergySBufs;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -99,7 +102,7 @@ block_energy_kernel(const __grid_constant__ CUtensorMap tm_k, const EnergyParams
         for (int s = 0; s < KST; ++s) { mbar_init(bar(L::B_KF + s), 1); mbar_init(bar(L::B_KE + s), 1); }
         for (int b = 0; b < SB; ++b) {
             mbar_init(bar(L::B_SF + b), 1);
-            mbar_init(bar(L::B_SE + b), kEnergySoftmaxThreads);
+            mbar_init(bar(L::B_SE + b), kEnergySoftmaxThreads / kEnergyGroups);   // one group per tile
         }
         mbar_init(bar(L::B_DRAIN), 1);
         *abort_flag = 0;
@@ -159,7 +162,7 @@ block_energy_kernel(const __grid_constant__ CUtensorMap tm_k, const EnergyParams
         }
     } else {
         // ===================== arithmetic (warps 2..9) ==================================
-        const int g = static_cast<int>(warp - 2) >> 2;      // column half of every tile
+        const int g = static_cast<int>(warp - 2) >> 2;      // group: tiles of parity g
         const int widx = static_cast<int>(warp) - 2;        // partial-sum table row
         const uint32_t q4 = warp & 3;
         const int r = static_cast<int>(q4 * 32 + lane);     // tile row == TMEM lane
@@ -199,14 +202,14 @@ block_energy_kernel(const __grid_constant__ CUtensorMap tm_k, const EnergyParams
             tc_fence_after();
             {
                 uint32_t raw[HC];
-                if constexpr (HC == 64) tmem_ld64_wait(tmem + lane_base + b * 128 + g * HC, raw);
-                else tmem_ld32_wait(tmem + lane_base + b * 128 + g * HC, raw);
+                if constexpr (HC == 128) tmem_ld128_wait(tmem + lane_base + b * 128, raw);
+                else tmem_ld64_wait(tmem + lane_base + b * 128, raw);
 #pragma unroll
                 for (int c = 0; c < HC; ++c) s[c] = __uint_as_float(raw[c]);
             }
             tc_fence_before();
             mbar_arrive(bar(L::B_SE + b));
-            const int valid = min(BLK, p.N - j * BLK) - g * HC;
+            const int valid = min(BLK, p.N - j * BLK);
             if (valid < HC) {
 #pragma unroll
                 for (int c = 0; c < HC; ++c)
@@ -230,9 +233,9 @@ block_energy_kernel(const __grid_constant__ CUtensorMap tm_k, const EnergyParams
 
         float lse2 = 0.f;
         if (two_pass) {
-            // ---- pass 1: exact running (max, sum) of this half of the row ----
+            // ---- pass 1: exact running (max, sum) of the row over this group's tiles ----
             float m_run = -INFINITY, l_run = 0.f;
-            for (int t = 0; t < nk; ++t) {
+            for (int t = g; t < nk; t += kEnergyGroups) {
                 float s[HC];
                 ok = load_tile(t, t, s);
                 if (!ok) break;
@@ -249,7 +252,7 @@ block_energy_kernel(const __grid_constant__ CUtensorMap tm_k, const EnergyParams
                 mx2 = fmaxf(mx2, s[HC - 2]);
                 mx3 = fmaxf(mx3, s[HC - 1]);
                 const float m_new = fmaxf(m_run, fmax3(mx0, mx1, fmaxf(mx2, mx3)) * sc);
-                // a half that has seen only masked columns keeps m = -inf and sum 0
+                // a group that has seen only masked columns keeps m = -inf and sum 0
                 const float m_sub = m_new == -INFINITY ? 0.f : m_new;
                 const float alpha = m_run == -INFINITY ? 0.f : ex2_approx(m_run - m_new);
                 l_run = l_run * alpha + exp_sum(s, m_sub);
@@ -271,13 +274,15 @@ block_energy_kernel(const __grid_constant__ CUtensorMap tm_k, const EnergyParams
             lse2 = p.lse_in[static_cast<size_t>(h) * p.Nq + qrow] * 1.4426950408889634f;
         }
 
-        // ---- pass 2: block sums, reduced per warp in batches of four key blocks ----
+        // ---- pass 2: block sums of this group's tiles (key block j is tile t0 + j), reduced
+        // per warp in batches of four ----
         const int t0 = two_pass ? nk : 0;
-        for (int jb = 0; ok && jb < nk; jb += 4) {
+        const int jg = (g - t0 % kEnergyGroups + kEnergyGroups) % kEnergyGroups;   // first own block
+        for (int jb = jg; ok && jb < nk; jb += 4 * kEnergyGroups) {
             float e4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-                const int j = jb + q;
+                const int j = jb + q * kEnergyGroups;
                 if (j < nk && ok) {
                     float s[HC];
                     ok = load_tile(t0 + j, j, s);
@@ -293,16 +298,18 @@ block_energy_kernel(const __grid_constant__ CUtensorMap tm_k, const EnergyParams
             if (lane == 0) {
 #pragma unroll
                 for (int q = 0; q < 4; ++q)
-                    if (jb + q < nk) red[widx * L::MAX_NK + jb + q] = e4[q];
+                    if (jb + q * kEnergyGroups < nk) red[widx * L::MAX_NK + jb + q * kEnergyGroups] = e4[q];
             }
         }
         named_bar_sync(kBarEnergy, kEnergySoftmaxThreads);   // every arithmetic warp gets here
         if (!*abort_flag) {
             float* dst = p.energy + (static_cast<size_t>(h) * p.nq + i) * nk;
             for (int j = static_cast<int>(threadIdx.x) - 64; j < nk; j += kEnergySoftmaxThreads) {
+                // the partials of block j come from the four warps of the group holding it
+                const int w0 = 4 * ((t0 + j) % kEnergyGroups);
                 float tot = 0.f;
 #pragma unroll
-                for (int w = 0; w < kEnergySoftmaxWarps; ++w) tot += red[w * L::MAX_NK + j];
+                for (int w = 0; w < 4; ++w) tot += red[(w0 + w) * L::MAX_NK + j];
                 dst[j] = p.accumulate ? dst[j] + tot : tot;
             }
         }
