@@ -369,11 +369,28 @@ select_mask_kernel(const __grid_constant__ SelectParams p) {
                     __syncwarp();
                     // G at each candidate's own pattern
                     uint64_t G0 = A, G1 = A;
-                    for (uint32_t x = 0; x < nc; ++x) {
-                        const uint4 e = cw[x];
-                        const uint64_t qe = (static_cast<uint64_t>(e.z) << 32) | e.y;
-                        if (e.x >= c0.x) G0 += qe;
-                        if (two && e.x >= c1.x) G1 += qe;
+                    // a loop per slot count; at MPL = 16 one loop with the second slot's test
+                    // inside measured faster (the two loops change its register allocation)
+                    constexpr bool kSplitLoop = MPL != 16;
+                    if (!kSplitLoop) {
+                        for (uint32_t x = 0; x < nc; ++x) {
+                            const uint4 e = cw[x];
+                            const uint64_t qe = (static_cast<uint64_t>(e.z) << 32) | e.y;
+                            if (e.x >= c0.x) G0 += qe;
+                            if (two && e.x >= c1.x) G1 += qe;
+                        }
+                    } else if (two) {
+                        for (uint32_t x = 0; x < nc; ++x) {
+                            const uint4 e = cw[x];
+                            const uint64_t qe = (static_cast<uint64_t>(e.z) << 32) | e.y;
+                            if (e.x >= c0.x) G0 += qe;
+                            if (e.x >= c1.x) G1 += qe;
+                        }
+                    } else {
+                        for (uint32_t x = 0; x < nc; ++x) {
+                            const uint4 e = cw[x];
+                            if (e.x >= c0.x) G0 += (static_cast<uint64_t>(e.z) << 32) | e.y;
+                        }
                     }
                     const uint32_t ustar =
                         warp_max_u32(max((v0 && G0 >= T) ? c0.x : 0u, (v1 && G1 >= T) ? c1.x : 0u));

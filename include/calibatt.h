@@ -90,8 +90,9 @@ calib_status calib_device_check(void* stream);
  *   q_rows   : NULL (query rows are the N tokens) or int32 [n_q] token indices in
  *              compacted order -- the anchor rows of a spatial-repetition head
  *              (calib_anchor_rows); then Nq = n_q and blocks are over that sequence.
- *   energy   : fp32 [H, ceil(Nq/B), ceil(N/B)].  accumulate != 0 adds to it (for the
- *              energy-sum aggregation over inputs); 0 overwrites.
+ *   energy   : fp32 [H, ceil(Nq/B), ceil(N/B)].  accumulate != 0 adds to it (the sum
+ *              over calibration inputs, which calib_energy_mean then divides by their
+ *              count); 0 overwrites.
  * P is never written to memory.  N <= 131072 (CALIB_ERR_UNSUPPORTED beyond: the per-block
  * partial sums of one query block are kept in shared memory). */
 calib_status calib_block_energy(const void* q, const void* k, const float* lse,
