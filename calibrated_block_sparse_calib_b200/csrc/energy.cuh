@@ -245,10 +245,12 @@ block_energy_kernel(const __grid_constant__ CUtensorMap tm_k, const EnergyParams
             return true;
         };
         // sum_c 2^(s_c * sc - m) with four independent packed accumulators.  The MUFU exp2
-        // unit bounds this pass, so one exponential in eight goes to the FMA pipe
-        // (exp2_poly2, relative error below 3e-6); 1/16 and 1/4 measured slower.  A masked
-        // column there adds about 2^-125 instead of 0, far below any energy's tolerance.
-        auto exp_sum = [&](const float (&s)[HC], float m) -> float {
+        // unit bounds this pass, so one pair of exponentials in every KP groups of four goes
+        // to the FMA pipe (exp2_poly2, relative error below 3e-6): a share of 1/(2 KP).
+        // Measured best: 1/4 in pass 1, whose max leaves the FMA pipe less busy, and 1/8 in
+        // pass 2 (1/16 and 1/4 there, and 1/2 in pass 1, were slower).  A masked column on
+        // the FMA pipe adds about 2^-125 instead of 0, far below any energy's tolerance.
+        auto exp_sum = [&](const float (&s)[HC], float m, const int KP) -> float {
             float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
 #pragma unroll
             for (int c = 0; c < HC; c += 4) {
@@ -257,7 +259,7 @@ block_energy_kernel(const __grid_constant__ CUtensorMap tm_k, const EnergyParams
                 ffma2(x2, x3, s[c + 2], s[c + 3], sc, sc, -m, -m);
                 fadd2(a0, a1, a0, a1, ex2_approx(x0), ex2_approx(x1));
                 float y2, y3;
-                if ((c / 4) % 4 == 3) {
+                if ((c / 4) % KP == KP - 1) {
                     exp2_poly2(y2, y3, x2, x3);
                 } else {
                     y2 = ex2_approx(x2);
@@ -292,7 +294,7 @@ block_energy_kernel(const __grid_constant__ CUtensorMap tm_k, const EnergyParams
                 // a group that has seen only masked columns keeps m = -inf and sum 0
                 const float m_sub = m_new == -INFINITY ? 0.f : m_new;
                 const float alpha = m_run == -INFINITY ? 0.f : ex2_approx(m_run - m_new);
-                l_run = l_run * alpha + exp_sum(s, m_sub);
+                l_run = l_run * alpha + exp_sum(s, m_sub, 2);
                 m_run = m_new;
             }
             xch[g * kTileM + r] = make_float2(m_run, l_run);
@@ -323,7 +325,7 @@ block_energy_kernel(const __grid_constant__ CUtensorMap tm_k, const EnergyParams
                 if (j < nk && ok) {
                     float s[HC];
                     ok = load_tile(t0 + j, j, s);
-                    if (ok && row_ok) e4[q] = exp_sum(s, lse2);
+                    if (ok && row_ok) e4[q] = exp_sum(s, lse2, 4);
                 }
             }
             if (!__all_sync(0xffffffffu, ok)) break;
