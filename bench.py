@@ -40,7 +40,7 @@ UNIT = "TFLOPS"
 # ncu capture of that launch (dram__bytes_read.sum + dram__bytes_write.sum), valid only for
 # the kernel sources it was taken on: reported as roofline.traffic while the source hashes
 # still match, else null.
-NCU_TRAFFIC = {("wan13b", "5de0933911ce", "4a81f0342eed"): 302_711_552 + 86_390_528}
+NCU_TRAFFIC = {("wan13b", "4d3844dc7507", "c7c3253ba1c1"): 302_891_520 + 86_448_896}
 
 # MUFU exp2 throughput of one SM: 4 lanes per clock in each of the 4 sub-partitions.
 MUFU_EX2_PER_CLK_SM = 16

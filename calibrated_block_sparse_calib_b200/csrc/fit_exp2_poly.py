@@ -1,4 +1,4 @@
-"""Fit of the degree-4 polynomial p(r) ~ 2^r on [-1/2, 1/2] used by exp2_poly2 (energy.cuh).
+"""Fit of the degree-4 polynomial p(r) ~ 2^r on [-1/2, 1/2] used by exp2_poly2 (ptx.cuh).
 
 Weighted least squares of the relative error at Chebyshev nodes, refined by Lawson
 reweighting towards the minimax (equioscillating) fit; then the coefficients are rounded

@@ -333,6 +333,33 @@ __device__ __forceinline__ void fadd2(float& d0, float& d1, float a0, float a1, 
         : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
 }
 
+// 2^x for a pair of floats on the FMA pipe instead of the MUFU unit (whose exp2
+// throughput, 16 per SM and clock, is the bound of the softmax-like passes).  Cody-Waite
+// style range reduction: n = x rounded to the nearest integer by adding and subtracting
+// 1.5 * 2^23, r = x - n in [-1/2, 1/2], 2^r by a degree-4 polynomial, then 2^n added to
+// the exponent field as an integer (the bits of 1.5 * 2^23 + n are 0x4B400000 + n, and
+// 0x4B400000 << 23 vanishes modulo 2^32).  The coefficients are a weighted least-squares
+// fit of 2^r on Chebyshev nodes refined towards minimax relative error (fit_exp2_poly.py
+// beside this file); maximum relative error 2.7e-6 in fp32.  Inputs are clamped to
+// [-125, 127] so the exponent arithmetic cannot wrap: results below 2^-125, and -inf
+// inputs (masked columns), come out as about 2^-125 instead of 0.
+__device__ __forceinline__ void exp2_poly2(float& y0, float& y1, float x0, float x1) {
+    constexpr float kMagic = 12582912.0f;   // 1.5 * 2^23
+    x0 = fminf(fmaxf(x0, -125.f), 127.f);
+    x1 = fminf(fmaxf(x1, -125.f), 127.f);
+    float t0, t1, n0, n1, r0, r1, p0, p1;
+    fadd2(t0, t1, x0, x1, kMagic, kMagic);
+    fadd2(n0, n1, t0, t1, -kMagic, -kMagic);
+    ffma2(r0, r1, n0, n1, -1.f, -1.f, x0, x1);
+    ffma2(p0, p1, 9.570096619427204e-3f, 9.570096619427204e-3f, r0, r1, 5.591785907745361e-2f,
+          5.591785907745361e-2f);
+    ffma2(p0, p1, p0, p1, r0, r1, 2.40247443318367e-1f, 2.40247443318367e-1f);
+    ffma2(p0, p1, p0, p1, r0, r1, 6.931217908859253e-1f, 6.931217908859253e-1f);
+    ffma2(p0, p1, p0, p1, r0, r1, 9.999992847442627e-1f, 9.999992847442627e-1f);
+    y0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+    y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     uint32_t r;
     // cvt packs its first source into the upper half: (hi, lo) puts `lo` in bits [0,16).

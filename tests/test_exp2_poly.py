@@ -1,6 +1,6 @@
-"""The FMA-pipe exp2 of the energy pass (exp2_poly2 in csrc/energy.cuh), checked on the CPU.
+"""The FMA-pipe exp2 of the energy pass (exp2_poly2 in csrc/ptx.cuh), checked on the CPU.
 
-The coefficients in energy.cuh must be the fp32 rounding of csrc/fit_exp2_poly.py's fit, and
+The coefficients in ptx.cuh must be the fp32 rounding of csrc/fit_exp2_poly.py's fit, and
 the routine -- round-to-nearest reduction by adding 1.5 * 2^23, a degree-4 Horner chain of
 fused multiply-adds, 2^n added to the exponent field as an integer -- is emulated in fp32
 and compared with float64 2^x.  No GPU is needed."""
@@ -23,7 +23,7 @@ def _fit_module():
 
 def _header_coefficients():
     """c0 .. c4 as written in exp2_poly2 (its Horner chain names c4 first, c0 last)."""
-    src = open(os.path.join(CSRC, "energy.cuh")).read()
+    src = open(os.path.join(CSRC, "ptx.cuh")).read()
     body = src[src.index("void exp2_poly2("):]
     body = body[:body.index("\n}\n")]
     lits = [float(x) for x in re.findall(r"([0-9]+\.[0-9]+e-?[0-9]+|[0-9]+\.[0-9]+)f", body)]
