@@ -132,9 +132,10 @@ __device__ __forceinline__ void red_shared_or(uint32_t addr, uint32_t v) {
 //   3. the blocks of bin k* (usually a few: a factor-of-sqrt(2) band of energies) are
 //      moved to shared memory in index order, two per lane, and each computes G at its own
 //      pattern from the others; u* is the largest pattern with G >= T.
-//   4. if no block outside bin k* can have q == v (checked by quantizing the two patterns
-//      just outside the bin), the blocks above bin k* are kept, and the bin's own blocks
-//      are decided in shared memory (q > v kept, then ties in index order).
+//   4. if no block outside bin k* can have q == v (true where q is exact from the pattern
+//      just below the bin up, else checked by quantizing the two patterns just outside the
+//      bin), the blocks above bin k* are kept, and the bin's own blocks are decided in
+//      shared memory (q > v kept, then ties in index order).
 // A row whose bin k* holds more than 64 blocks, or whose ties may cross the bin's edges,
 // takes the exact bisection over the bit patterns instead (at most 31 steps over all of the
 // row's elements).
