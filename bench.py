@@ -617,9 +617,10 @@ def main():
         if world > 1:
             ms_serial = max_over_ranks(ms_serial, dist, dev)
         nb = q.numel() * q.element_size()
-        # sparse_attn_fwd_host: per chunk of 2 heads, the host -> device copies of the next
-        # chunk and the device -> host copy of the previous one overlap the attention
-        hpc = 2
+        # sparse_attn_fwd_host: per chunk of 3 heads (the last chunk's heads one at a time), the
+        # host -> device copies of the next chunk and the device -> host copy of the previous
+        # one overlap the attention
+        hpc = 3
         staging = ops.HostStaging(qd, kd, vd, out)
         geom = (rep, s.F, s.Hl, s.Wl, s.n_text, stride) if any(rep) else None
         ms_e2e = _time_calls(lambda: ops.sparse_attn_fwd_host(qh, kh, vh, bl, staging=staging, out=oh,

@@ -226,8 +226,11 @@ calib_status host_pipeline(const AttnCall& c, const void* q_host, const void* k_
     // the copy streams start after the work already queued on the caller's stream
     if (cudaStreamWaitEvent(sin, start, 0) != cudaSuccess || cudaStreamWaitEvent(sout, start, 0) != cudaSuccess)
         return CALIB_ERR_CUDA;
-    for (int h0 = 0; h0 < H; h0 += hpc) {
-        const int h1 = h0 + hpc < H ? h0 + hpc : H;
+    // The step ends with the last chunk's kernel and copy-back after the last host-to-device
+    // copy, so when there are several chunks the last chunk's heads go one per chunk.
+    for (int h0 = 0, h1 = 0; h0 < H; h0 = h1) {
+        h1 = h0 + hpc < H ? h0 + hpc : H;
+        if (h1 == H && h0 > 0) h1 = h0 + 1;
         const size_t off = static_cast<size_t>(h0) * in_head, len = static_cast<size_t>(h1 - h0) * in_head;
         // one copy per tensor and chunk
         if (cudaMemcpyAsync(static_cast<char*>(q_dev) + off, static_cast<const char*>(q_host) + off, len,

@@ -256,6 +256,9 @@ calib_status sparse_attn_fwd(const void* q, const void* k, const void* v, void* 
  *   heads_per_chunk >= 1.  Chunks follow the work list, which must then hold each head's nq
  *                items contiguously in head order (as calib_build_schedule writes it);
  *                with list->work == NULL or n_work != H*nq the call runs as one chunk.
+ *                When there are several chunks, the heads of the last one go one head per
+ *                chunk: the kernel and copy-back after the last host-to-device copy are
+ *                then one head's.
  *   h2d_stream, d2h_stream : copy streams (NULL: `stream`, no overlap).
  * Ordering: the copies start after the work already queued on `stream`, and `stream` is
  * ordered after the last copy of O, so synchronising `stream` makes o_host complete.
