@@ -165,11 +165,13 @@ def _hard_rows(rng, H, nq, nk):
     return e
 
 
-@pytest.mark.parametrize("nk", [1, 2, 33, 64, 100, 256, 591, 1024])
+@pytest.mark.parametrize("nk", [1, 2, 33, 64, 100, 101, 255, 256, 300, 350, 591, 600, 999, 1024])
 def test_select_batched_bit_exact(nk):
     """One launch over nb entries, each at its own tau, with shared forced blocks, per-entry
     masks and vote counts: every entry's mask equals the oracle's selection of that entry,
-    and the counts equal the sum of the masks."""
+    and the counts equal the sum of the masks.  The widths cover every energies-per-lane
+    count (2, 4, 8, 16, 20, 32) with rows that are 16-byte aligned (nk % 4 == 0: vector
+    loads) and rows that are not (staged through shared memory)."""
     rng = np.random.default_rng(1000 + nk)
     taus = [1e-7, 0.5, 0.9, 0.95, 0.99, 1.0]
     H, nq = 2, 5
