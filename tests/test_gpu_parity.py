@@ -358,7 +358,8 @@ def test_energy_tiny_all_inputs(tiny_inputs):
         check_energy(got, ref, wl.shape.N, B)
 
 
-@pytest.mark.parametrize("D,B,geom", [(128, 128, (5, 10, 20)), (128, 64, (3, 9, 11)), (64, 128, (2, 13, 17))])
+@pytest.mark.parametrize("D,B,geom", [(128, 128, (5, 10, 20)), (128, 64, (3, 9, 11)), (64, 128, (2, 13, 17)),
+                                      (128, 128, (3, 9, 13)), (128, 128, (1, 8, 10))])
 def test_energy_ragged(D, B, geom):
     wl = _shape(2, D, *geom, B)
     q, k, _ = _inputs(wl, seed=100 + D + B)
